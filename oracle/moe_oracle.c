@@ -1,0 +1,256 @@
+/*
+ * moe_oracle.c -- CPU oracle for MoE token dispatch and combine.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the bench's
+ * CPU-baseline leg may load this file's library.  The product path never does;
+ * it shares no code, header or table with this file.
+ *
+ * This is a plain, slow, single-threaded statement of what the path computes,
+ * written from the pages, with no blocking, fusion or reordering:
+ *
+ *   Dispatch ("Enabling trillion-parameter models on AWS EFA", sections
+ *   "Introdução" and "MoE all-to-all sobre EFA"): take the tokens and each
+ *   token's experts and group the tokens by expert.  Section "Buffers de Envio e
+ *   Recebimento" and section "Despacho e Combinação" fix how: count the tokens
+ *   per expert, take the cumulative sum of the counts as offsets, and pack each
+ *   expert's tokens contiguously from its offset.  Inside an expert's segment the
+ *   tokens are kept in (token, k) order, so the dispatch is a stable counting
+ *   sort of the T*k routing entries by expert id.
+ *
+ *   Block fp8 ("Lower latency and higher throughput with multi-node DeepSeek
+ *   deployment", section "Quantização"; the EFA article, section "Avaliação":
+ *   "block-scaled fp8 dispatch"): one fp32 scale per 128-element activation
+ *   vector, computed from that vector.  Scale = amax / 448 (448 is the largest
+ *   finite e4m3 value), codes = e4m3(x / scale), rounded to nearest with ties to
+ *   even and saturated to +-448.
+ *
+ *   Combine (EFA article, sections "Introdução", "Buffers de Envio e
+ *   Recebimento" and "Despacho e Combinação"; DeepSeek article, section
+ *   "Paralelismo de Especialistas"): gather each token's processed rows back and
+ *   form the routing-weighted sum.  Evaluated here in fp64.
+ *
+ * Readings where the pages are silent:
+ *   - weights are used as given (weighted sum, no division by their total);
+ *   - an expert id outside [0, E) is dropped and flagged (error bit 1);
+ *   - an entry whose slot would fall at or beyond the receive capacity is
+ *     dropped and flagged (error bit 2); its slot is -1;
+ *   - receive rows that hold no entry (padding, unused capacity) have
+ *     recv_src = -1, and their payload is left untouched;
+ *   - an all-zero 128-block gets scale 0 and all codes +0.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+#include <stdlib.h>
+
+#define ORACLE_BAD_INDEX 1
+#define ORACLE_CAPACITY 2
+
+/* A bf16 value is the upper 16 bits of an IEEE binary32. */
+static float bf16_to_float(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/*
+ * e4m3 ("E4M3", OCP 8-bit floating point specification): 1 sign bit, 4 exponent
+ * bits with bias 7, 3 mantissa bits.  No infinities; S.1111.111 is NaN, so the
+ * largest finite magnitude is S.1111.110 = 1.75 * 2^8 = 448.  Exponent field 0
+ * holds the subnormals m * 2^-9 (m = 0..7); field f >= 1 holds (1 + m/8) * 2^(f-7).
+ *
+ * Conversion of a finite float v: round |v| to the nearest point of that grid
+ * (ties to the point whose mantissa is even), clamp the result to 448, keep the
+ * sign of v.
+ */
+uint8_t oracle_e4m3_from_float(float v)
+{
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    double a = fabs((double)v);
+
+    /* Spacing of the grid around a: 2^-9 below the smallest normal 2^-6,
+     * else 2^(floor(log2 a) - 3) (three mantissa bits). */
+    double step;
+    if (a < 0x1p-6) {
+        step = 0x1p-9;
+    } else {
+        int e;
+        frexp(a, &e);              /* a = f * 2^e with f in [0.5, 1) */
+        step = ldexp(1.0, (e - 1) - 3);
+    }
+    /* a/step is exact (step is a power of two); nearbyint rounds ties to even
+     * in the default rounding mode, and an even multiple of the step is a code
+     * with an even mantissa. */
+    double q = nearbyint(a / step) * step;
+    if (q > 448.0)
+        q = 448.0;
+
+    uint8_t bits;
+    if (q < 0x1p-6) {
+        bits = (uint8_t)(q / 0x1p-9);          /* field 0, mantissa q/2^-9 */
+    } else {
+        int e;
+        frexp(q, &e);
+        int unbiased = e - 1;                  /* q = (1 + m/8) * 2^unbiased */
+        int m = (int)((q / ldexp(1.0, unbiased) - 1.0) * 8.0);
+        bits = (uint8_t)(((unbiased + 7) << 3) | m);
+    }
+    return (uint8_t)(sign | bits);
+}
+
+/*
+ * Quantise one token's hidden vector (H bf16 values, H a multiple of 128) to
+ * e4m3 codes with one fp32 scale per 128-element block.
+ */
+static void quantise_row_fp8(const uint16_t *x, int32_t H, uint8_t *codes, float *scales)
+{
+    for (int32_t b = 0; b < H / 128; ++b) {
+        float amax = 0.0f;
+        for (int32_t i = 0; i < 128; ++i) {
+            float v = fabsf(bf16_to_float(x[b * 128 + i]));
+            if (v > amax)
+                amax = v;
+        }
+        if (amax == 0.0f) {
+            scales[b] = 0.0f;
+            for (int32_t i = 0; i < 128; ++i)
+                codes[b * 128 + i] = 0x00;
+            continue;
+        }
+        float scale = amax / 448.0f;                     /* binary32, round to nearest */
+        scales[b] = scale;
+        for (int32_t i = 0; i < 128; ++i) {
+            float q = bf16_to_float(x[b * 128 + i]) / scale;  /* binary32, round to nearest */
+            codes[b * 128 + i] = oracle_e4m3_from_float(q);
+        }
+    }
+}
+
+/* Rows an expert segment takes: its count, rounded up to a multiple of 128
+ * when padding is on. */
+static int64_t padded(int64_t count, int32_t pad128)
+{
+    return pad128 ? (count + 127) / 128 * 128 : count;
+}
+
+/*
+ * Dispatch.  Inputs: x[T,H] bf16 bits, topk_idx[T,k].  Outputs (all written):
+ *   expert_count[E], expert_offset[E+1], rank_offset[R+1], slot[T,k],
+ *   recv_src[rows_cap]; payload rows recv_x[slot] (bf16 bits, or e4m3 codes
+ *   with recv_scale[slot, H/128]) for every kept entry.
+ * Returns the OR of the error bits.
+ */
+int32_t oracle_dispatch(int32_t T, int32_t H, int32_t k, int32_t E, int32_t R,
+                        int32_t fp8, int32_t pad128, int64_t rows_cap,
+                        const uint16_t *x, const int32_t *topk_idx,
+                        void *recv_x, float *recv_scale,
+                        int32_t *expert_count, int32_t *expert_offset,
+                        int32_t *rank_offset, int32_t *recv_src, int32_t *slot)
+{
+    int32_t err = 0;
+
+    /* 1. Per-expert token counts. */
+    for (int32_t e = 0; e < E; ++e)
+        expert_count[e] = 0;
+    for (int32_t t = 0; t < T; ++t)
+        for (int32_t j = 0; j < k; ++j) {
+            int32_t e = topk_idx[(int64_t)t * k + j];
+            if (e < 0 || e >= E)
+                err |= ORACLE_BAD_INDEX;
+            else
+                expert_count[e] += 1;
+        }
+
+    /* 2. Offsets: cumulative sum of the (optionally padded) counts. */
+    expert_offset[0] = 0;
+    for (int32_t e = 0; e < E; ++e)
+        expert_offset[e + 1] = (int32_t)(expert_offset[e] + padded(expert_count[e], pad128));
+
+    /* 3. Rank r hosts experts [r*E/R, (r+1)*E/R); its buffer starts where its
+     *    first expert's segment starts. */
+    for (int32_t r = 0; r <= R; ++r)
+        rank_offset[r] = expert_offset[(int64_t)r * (E / R)];
+
+    /* 4. Slots: walk the entries in (token, k) order; each expert hands out the
+     *    next row of its segment. */
+    for (int64_t i = 0; i < rows_cap; ++i)
+        recv_src[i] = -1;
+    int32_t *cursor = (int32_t *)malloc(sizeof(int32_t) * (size_t)(E > 0 ? E : 1));
+    for (int32_t e = 0; e < E; ++e)
+        cursor[e] = expert_offset[e];
+    for (int32_t t = 0; t < T; ++t)
+        for (int32_t j = 0; j < k; ++j) {
+            int64_t i = (int64_t)t * k + j;
+            int32_t e = topk_idx[i];
+            if (e < 0 || e >= E) {
+                slot[i] = -1;
+                continue;
+            }
+            int32_t s = cursor[e]++;
+            if (s >= rows_cap) {
+                err |= ORACLE_CAPACITY;
+                slot[i] = -1;
+                continue;
+            }
+            slot[i] = s;
+            recv_src[s] = (int32_t)i;
+        }
+    free(cursor);
+
+    /* 5. Payload: the token's row (or its e4m3 codes and scales) to every slot. */
+    int32_t nb = H / 128;
+    uint8_t *codes = NULL;
+    float *scales = NULL;
+    if (fp8) {
+        codes = (uint8_t *)malloc((size_t)H);
+        scales = (float *)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
+    }
+    for (int32_t t = 0; t < T; ++t) {
+        const uint16_t *xt = x + (int64_t)t * H;
+        if (fp8)
+            quantise_row_fp8(xt, H, codes, scales);
+        for (int32_t j = 0; j < k; ++j) {
+            int32_t s = slot[(int64_t)t * k + j];
+            if (s < 0)
+                continue;
+            if (fp8) {
+                memcpy((uint8_t *)recv_x + (int64_t)s * H, codes, (size_t)H);
+                memcpy(recv_scale + (int64_t)s * nb, scales, sizeof(float) * (size_t)nb);
+            } else {
+                memcpy((uint16_t *)recv_x + (int64_t)s * H, xt, sizeof(uint16_t) * (size_t)H);
+            }
+        }
+    }
+    free(codes);
+    free(scales);
+    return err;
+}
+
+/*
+ * Combine: y[t,h] = sum_j topk_w[t,j] * expert_out[slot[t,j], h], in fp64,
+ * j ascending.  Entries with slot -1 (dropped at dispatch) contribute nothing.
+ */
+void oracle_combine(int32_t T, int32_t H, int32_t k, const int32_t *slot,
+                    const float *topk_w, const uint16_t *expert_out, double *y)
+{
+    for (int32_t t = 0; t < T; ++t)
+        for (int32_t h = 0; h < H; ++h) {
+            double acc = 0.0;
+            for (int32_t j = 0; j < k; ++j) {
+                int32_t s = slot[(int64_t)t * k + j];
+                if (s < 0)
+                    continue;
+                acc += (double)topk_w[(int64_t)t * k + j] *
+                       (double)bf16_to_float(expert_out[(int64_t)s * H + h]);
+            }
+            y[(int64_t)t * H + h] = acc;
+        }
+}
+
+/* The block quantiser alone, for one row: exposed for the tests' pins. */
+void oracle_quantise_row_fp8(const uint16_t *x, int32_t H, uint8_t *codes, float *scales)
+{
+    quantise_row_fp8(x, H, codes, scales);
+}
