@@ -1,0 +1,414 @@
+"""Benchmark of MoE dispatch + combine on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path -- routing metadata, dispatch payload
+(bf16 copy or fp8 block quantisation) and combine -- over one batch of
+synthetic inputs already resident in HBM.  Every step starts from a flushed L2
+(a 2x-L2 memset outside the timed events), and dispatch and combine replay as
+CUDA graphs, so the events time the GPU work and not Python.
+
+`value` is the achieved HBM throughput of the step: the algorithmic bytes of
+dispatch + combine (x read once, k payload rows written per token, metadata;
+combine reads k rows per token and writes y; padding rows are not counted)
+divided by the step time, summed over ranks.  Under torchrun every rank runs
+its own batch (weak scaling) and the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+DEFAULT_WORKLOAD = "dsv3_decode"
+METRIC = "dispatch+combine µs and achieved HBM GB/s (% of B200 peak) per config"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def algorithmic_bytes(T, H, E, R, k, fp8):
+    """(dispatch bytes, combine bytes) the method must move, padding excluded."""
+    S = T * k
+    nb = H // 128
+    dispatch = T * H * 2 + S * 4 + (S * H + S * nb * 4 if fp8 else S * H * 2)
+    dispatch += E * 4 + (E + 1) * 4 + (R + 1) * 4 + 2 * S * 4
+    combine = S * H * 2 + 2 * S * 4 + T * H * 2
+    return dispatch, combine
+
+
+def combine_kernel_bytes(T, H, k):
+    S = T * k
+    return S * H * 2 + 2 * S * 4 + T * H * 2
+
+
+def measured_peak():
+    p = os.path.join(HERE, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest(name):
+    p = os.path.join(HERE, "combine_route_meta_b200", "csrc", name)
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel_file, workload):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel is unchanged."""
+    p = os.path.join(HERE, "profiles", "dram_traffic.json")
+    try:
+        with open(p) as f:
+            rec = json.load(f)
+        e = rec[kernel_file][workload]
+        if e["source_sha256_16"] != source_digest(kernel_file):
+            return None
+        return int(e["bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+# ---- CPU oracle arm ---------------------------------------------------------------
+
+def oracle_sample_workload(w):
+    """A bounded sample of the workload for the CPU oracle: fewer tokens, same routing recipe."""
+    import dataclasses
+    t_sample = min(w.T, 512 if w.H >= 4096 else w.T)
+    return dataclasses.replace(w, T=t_sample)
+
+
+class OracleRun:
+    """The CPU oracle on a bounded sample of the workload, inputs prepared once."""
+
+    def __init__(self, w):
+        import oracle
+        from workloads import make_expert_out, make_inputs
+        self.oracle = oracle
+        oracle.build()
+        self.ws = ws = oracle_sample_workload(w)
+        _, self.x, self.idx, self.wts = make_inputs(ws)
+        self.cap = oracle.rows_capacity(ws.T, ws.k, ws.E, ws.pad128)
+        self.eo = None if ws.identity_experts else make_expert_out(ws, self.cap)
+        db, cb = algorithmic_bytes(ws.T, ws.H, ws.E, ws.R, ws.k, ws.fp8)
+        self.bytes = db + cb
+        self.desc = (f"oracle dispatch+combine (single-threaded C, fp64 combine) on the first "
+                     f"{ws.T} of {w.T} tokens of {w.name}")
+
+    def once(self):
+        """Seconds for one dispatch + combine."""
+        ws, o = self.ws, self.oracle
+        t0 = time.perf_counter()
+        d = o.dispatch(self.x, self.idx, E=ws.E, R=ws.R, fp8=ws.fp8, pad128=ws.pad128,
+                       rows_cap=self.cap)
+        o.combine(d["slot"], self.wts, d["recv_x"] if self.eo is None else self.eo)
+        return time.perf_counter() - t0
+
+
+def time_oracle(w, budget_s=10.0, max_reps=50):
+    """(GB/s of algorithmic bytes, description) of the oracle on a bounded sample."""
+    run = OracleRun(w)
+    times = []
+    t_end = time.perf_counter() + budget_s
+    while len(times) < max_reps and (not times or time.perf_counter() < t_end):
+        times.append(run.once())
+    med = statistics.median(times)
+    return run.bytes / med / 1e9, f"{run.desc}, median of {len(times)} runs"
+
+
+# ---- GPU arm ----------------------------------------------------------------------------
+
+def run_gpu(args, rank, world):
+    import torch
+    import combine_route_meta_b200 as moe
+    from workloads import WORKLOADS, make_expert_out, make_inputs
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    import dataclasses
+    w = dataclasses.replace(w, seed=w.seed + rank)
+    _, x, idx, wts = make_inputs(w)
+    cfg = moe.make_config(w.H, w.k, w.E, w.R, w.fp8, w.pad128)
+    buf = moe.Buffers(cfg, w.T, dev)
+    eo_host = make_expert_out(w, buf.rows_cap)
+
+    def bf16_dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    xd, idd, wd = bf16_dev(x), torch.from_numpy(idx).to(dev), torch.from_numpy(wts).to(dev)
+    eo = buf.recv_x if w.identity_experts else bf16_dev(eo_host)
+    if w.identity_experts and w.fp8:
+        raise SystemExit("identity experts need a bf16 dispatch")
+    y = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev)
+
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def do_dispatch():
+        moe.dispatch_into(buf, xd, idd, wd, stream=stream)
+
+    def do_combine():
+        moe.combine_into(buf.handle_c, eo, y, buf.err, stream=stream)
+
+    # warm-up (also loads the kernels) and graph capture on a side stream
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            do_dispatch()
+            do_combine()
+    stream.synchronize()
+    g_disp, g_comb = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_disp, stream=stream):
+        do_dispatch()
+    with torch.cuda.graph(g_comb, stream=stream):
+        do_combine()
+    if moe.check(stream) != 0:
+        raise RuntimeError("device error during warm-up")
+
+    launches_per_step = (1 if moe.workspace_bytes(cfg, w.T) == 0 else 3) + 1 + 1
+
+    def step(evs):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+            torch.cuda._sleep(20_000)  # lets the host queue the step before the GPU reaches it
+            evs[0].record(stream)
+            g_disp.replay()
+            evs[1].record(stream)
+            g_comb.replay()
+            evs[2].record(stream)
+
+    for _ in range(args.warmup):
+        step([torch.cuda.Event(enable_timing=True) for _ in range(3)])
+    torch.cuda.synchronize()
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    all_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for evs in all_evs:
+        step(evs)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+
+    disp_ms = [a.elapsed_time(b) for a, b, _ in all_evs]
+    comb_ms = [b.elapsed_time(c) for _, b, c in all_evs]
+    step_ms = [a.elapsed_time(c) for a, _, c in all_evs]
+    bits = moe.check(stream)
+    if bits:
+        raise RuntimeError(f"device error bits {bits} during timing")
+
+    total_ms = sum(step_ms)
+    if dist is not None:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # end-to-end through the public API with host buffers: H2D of the step's inputs,
+    # dispatch, combine, D2H of y, every step
+    pin = dict(pin_memory=True)
+    x_h = torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).pin_memory()
+    idx_h = torch.from_numpy(idx).pin_memory()
+    w_h = torch.from_numpy(wts).pin_memory()
+    eo_h = (None if w.identity_experts else
+            torch.from_numpy(np.ascontiguousarray(eo_host).view(np.int16)).view(torch.bfloat16).pin_memory())
+    y_h = torch.empty((w.T, w.H), dtype=torch.bfloat16, **pin)
+    h2d = x_h.numel() * 2 + idx_h.numel() * 4 + w_h.numel() * 4 + (0 if eo_h is None else eo_h.numel() * 2)
+    d2h = y_h.numel() * 2
+    e2e_steps = max(3, min(args.steps, 20))
+    e2e_ms = []
+    for i in range(args.warmup + e2e_steps):
+        with torch.cuda.stream(stream):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            xd.copy_(x_h, non_blocking=True)
+            idd.copy_(idx_h, non_blocking=True)
+            wd.copy_(w_h, non_blocking=True)
+            if eo_h is not None:
+                eo.copy_(eo_h, non_blocking=True)
+            do_dispatch()
+            do_combine()
+            y_h.copy_(y, non_blocking=True)
+            e1.record(stream)
+        e1.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(e0.elapsed_time(e1))
+
+    return dict(w=w, buf=buf, disp_ms=disp_ms, comb_ms=comb_ms, step_ms=step_ms,
+                total_ms=total_ms, clocks=clocks, launches_per_step=launches_per_step,
+                e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, moe=moe)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    from workloads import WORKLOADS
+    w0 = WORKLOADS[args.workload]
+    peak, peak_kind = measured_peak()
+
+    if args.impl == "reference":
+        # The reference arm is the CPU oracle, timed on this host's cores (rank 0 only).
+        if rank != 0:
+            return
+        run = OracleRun(w0)
+        per_step = [run.once() for _ in range(args.warmup + args.steps)][args.warmup:]
+        total = sum(per_step)
+        g = run.bytes * args.steps / total / 1e9
+        ms = total / args.steps * 1e3
+        desc = f"{run.desc}, {args.steps} timed runs"
+        line = {
+            "impl": "reference", "metric": METRIC, "value": round(g, 3), "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "T": w0.T, "H": w0.H, "E": w0.E, "R": w0.R,
+                       "k": w0.k, "payload": "fp8" if w0.fp8 else "bf16", "pad128": w0.pad128},
+            "cpu_baseline": {"value": round(g, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": round(g, 3), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    r = run_gpu(args, rank, world)
+    w, moe = r["w"], r["moe"]
+    db, cb = algorithmic_bytes(w.T, w.H, w.E, w.R, w.k, w.fp8)
+    step_bytes = db + cb
+    ms_per_step = r["total_ms"] / args.steps
+    value = step_bytes * world / (ms_per_step * 1e-3) / 1e9
+
+    disp_us = statistics.median(r["disp_ms"]) * 1e3
+    comb_us = statistics.median(r["comb_ms"]) * 1e3
+    comb_mean_s = statistics.mean(r["comb_ms"]) * 1e-3
+    ck_bytes = combine_kernel_bytes(w.T, w.H, w.k)
+    achieved = ck_bytes / comb_mean_s / 1e9
+    roofline = {"bound": "hbm", "kernel": "combine_rows", "achieved": round(achieved, 1),
+                "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                "frac": round(achieved / peak, 4),
+                "traffic": recorded_traffic("combine.cuh", w.name),
+                "algorithmic_bytes": ck_bytes}
+    e2e_s = statistics.median(r["e2e_ms"]) * 1e-3
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": w.name, "T": w.T, "H": w.H, "E": w.E, "R": w.R, "k": w.k,
+                   "payload": "fp8 e4m3 + fp32 scale per 128" if w.fp8 else "bf16",
+                   "pad128": w.pad128, "combine": "bf16 out, fp32 accumulate",
+                   "l2": "flushed (2x L2 memset) before every step", "graphs": True,
+                   "parallelism": f"replicas x{world}"},
+        "dispatch_us": round(disp_us, 2), "combine_us": round(comb_us, 2),
+        "total_us": round(ms_per_step * 1e3, 2),
+        "pct_of_peak": round(100 * step_bytes / (ms_per_step * 1e-3) / 1e9 / peak, 2),
+        "bytes_per_step": {"dispatch": db, "combine": cb},
+        "roofline": roofline,
+        "e2e": {"value": round(step_bytes / e2e_s / 1e9, 3), "unit": "GB/s",
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+                "ms_per_step": round(e2e_s * 1e3, 4)},
+        "gpu_launches": r["launches_per_step"] * args.steps,
+        "clocks": r["clocks"],
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        g, desc = time_oracle(w0)
+        line["cpu_baseline"] = {"value": round(g, 4), "unit": "GB/s", "cores": 1,
+                                "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,287 @@
+// Routing metadata: per-expert counts, offsets and deterministic slots.
+//
+// "Enabling trillion-parameter models on AWS EFA", section "Despacho e
+// Combinação": the dispatch first counts the tokens routed to each expert
+// (atomic accumulation in shared memory), then takes the cumulative sum of the
+// counts to find where each expert's tokens are packed contiguously; section
+// "Buffers de Envio e Recebimento" asks for contiguous packing so that no
+// private per-sender space is needed.  The order inside an expert's segment is
+// fixed here as (token, k) ascending, which makes slot assignment a stable
+// counting sort of the S = T*k routing entries by expert id.
+//
+// GPU design.  Entries are processed in rounds of one entry per thread.  In a
+// round, lanes of a warp holding the same expert find each other with
+// __match_any_sync: the lowest such lane does one shared-memory update for the
+// whole group (so a skewed routing where most tokens pick one expert does not
+// serialise on one counter), and a lane's rank inside the group is the
+// population count of the group's lanes below it.  A lane's slot is then
+//   cursor[e]                          (rows handed out to e by earlier rounds)
+// + sum over lower warps of their group sizes for e   (this round)
+// + rank inside its own warp's group.
+// That is exactly the stable order, with no sort and no global atomics.
+//
+// Two launch shapes:
+//  - small batches (S <= kSingleBlockEntries): one CTA does counts, scan and
+//    slots in shared memory (one launch, no scratch);
+//  - large batches: tiles of kTileEntries entries.  (1) each CTA counts its
+//    tile into scratch tile_hist[tile][E]; (2) one CTA turns those into
+//    per-tile prefixes, the counts and the offsets; (3) each CTA re-reads its
+//    tile and assigns slots from offset[e] + tile prefix.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kMetaThreads = 512;
+constexpr int kMetaWarps = kMetaThreads / kWarp;
+constexpr int kTileEntries = 2048;
+constexpr int kSingleBlockEntries = 4096;
+
+struct MetaArgs {
+    const int32_t *topk_idx;
+    int64_t S; // T*k routing entries
+    int32_t k, E, R, pad128;
+    int64_t rows_cap;
+    int32_t *expert_count;  // [E]
+    int32_t *expert_offset; // [E+1]
+    int32_t *rank_offset;   // [R+1]
+    int32_t *slot;          // [S]
+    int32_t *recv_src;      // [rows_cap]
+    int32_t *err;
+};
+
+// Expert id of entry i, or -1 for no entry (past the end, or out of range).
+__device__ __forceinline__ int32_t entry_expert(const MetaArgs &a, int64_t i, bool flag_bad)
+{
+    if (i >= a.S)
+        return -1;
+    int32_t e = __ldg(a.topk_idx + i);
+    if (e < 0 || e >= a.E) {
+        if (flag_bad)
+            raise_error(a.err, MOE_DEV_BAD_INDEX);
+        return -1;
+    }
+    return e;
+}
+
+// Adds the entries [begin, end) into hist[E] (shared memory).
+__device__ __forceinline__ void block_count(const MetaArgs &a, int64_t begin, int64_t end,
+                                            int32_t *hist)
+{
+    const unsigned lane = lane_id();
+    for (int64_t base = begin; base < end; base += kMetaThreads) {
+        int64_t i = base + threadIdx.x;
+        int32_t e = i < end ? entry_expert(a, i, true) : -1;
+        unsigned peers = __match_any_sync(kFullMask, e);
+        if (e >= 0 && lane == (unsigned)(__ffs(peers) - 1))
+            atomicAdd(&hist[e], __popc(peers));
+    }
+}
+
+// Exclusive scan of the (optionally 128-padded) counts in shared memory:
+// off[e] = sum_{e' < e} seg(e'), off[E] = total.  `cnt` and `off` may not alias.
+// Uses the whole block; ends with a barrier.
+__device__ void block_offsets(const int32_t *cnt, int32_t *off, int32_t E, int32_t pad128)
+{
+    __shared__ int32_t warp_sums[kMetaWarps];
+    __shared__ int32_t carry;
+    if (threadIdx.x == 0)
+        carry = 0;
+    __syncthreads();
+    const unsigned lane = lane_id(), warp = threadIdx.x / kWarp;
+    for (int32_t base = 0; base < E; base += kMetaThreads) {
+        int32_t e = base + threadIdx.x;
+        int32_t v = 0;
+        if (e < E) {
+            v = cnt[e];
+            if (pad128)
+                v = (v + 127) / 128 * 128;
+        }
+        int32_t incl = v;
+#pragma unroll
+        for (int d = 1; d < kWarp; d <<= 1) {
+            int32_t n = __shfl_up_sync(kFullMask, incl, d);
+            if (lane >= (unsigned)d)
+                incl += n;
+        }
+        if (lane == kWarp - 1)
+            warp_sums[warp] = incl;
+        __syncthreads();
+        int32_t before = carry;
+        for (unsigned w = 0; w < warp; ++w)
+            before += warp_sums[w];
+        if (e < E)
+            off[e] = before + incl - v;
+        __syncthreads();
+        if (threadIdx.x == kMetaThreads - 1)
+            carry = before + incl;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0)
+        off[E] = carry;
+    __syncthreads();
+}
+
+// Assigns slots to entries [begin, end) in order.  cursor[e] (shared) holds the
+// first free row of expert e for this range and is advanced; wcnt is
+// [kMetaWarps][E] shared scratch that must be zero on entry and is zero on exit.
+__device__ __forceinline__ void block_assign(const MetaArgs &a, int64_t begin, int64_t end,
+                                             int32_t *cursor, int32_t *wcnt)
+{
+    const unsigned lane = lane_id(), warp = threadIdx.x / kWarp;
+    for (int64_t base = begin; base < end; base += kMetaThreads) {
+        int64_t i = base + threadIdx.x;
+        int32_t e = i < end ? entry_expert(a, i, false) : -1;
+        unsigned peers = __match_any_sync(kFullMask, e);
+        unsigned leader = __ffs(peers) - 1;
+        int32_t rank = __popc(peers & lanemask_lt());
+        int32_t group = __popc(peers);
+        bool lead = e >= 0 && lane == leader;
+        if (lead)
+            wcnt[warp * a.E + e] = group;
+        __syncthreads();
+        int32_t first = 0;
+        if (lead) {
+            first = cursor[e];
+            for (unsigned w = 0; w < warp; ++w)
+                first += wcnt[w * a.E + e];
+        }
+        first = __shfl_sync(kFullMask, first, leader);
+        __syncthreads();
+        if (lead) {
+            atomicAdd(&cursor[e], group);
+            wcnt[warp * a.E + e] = 0;
+        }
+        if (i < end) {
+            int32_t s = -1;
+            if (e >= 0) {
+                int64_t row = (int64_t)first + rank;
+                if (row < a.rows_cap) {
+                    s = (int32_t)row;
+                    a.recv_src[row] = (int32_t)i;
+                } else {
+                    raise_error(a.err, MOE_DEV_CAPACITY);
+                }
+            }
+            a.slot[i] = s;
+        }
+        __syncthreads();
+    }
+}
+
+// recv_src = -1 on rows that hold no entry: each expert's padding, and the rows
+// from expert_offset[E] to rows_cap.  Work is split over `nblk` blocks.
+__device__ __forceinline__ void block_fill_unused(const MetaArgs &a, const int32_t *cnt,
+                                                  const int32_t *off, int blk, int nblk)
+{
+    for (int32_t e = blk; e < a.E; e += nblk) {
+        int64_t lo = (int64_t)off[e] + cnt[e];
+        int64_t hi = off[e + 1] < a.rows_cap ? off[e + 1] : a.rows_cap;
+        for (int64_t r = lo + threadIdx.x; r < hi; r += kMetaThreads)
+            a.recv_src[r] = -1;
+    }
+    for (int64_t r = (int64_t)off[a.E] + (int64_t)blk * kMetaThreads + threadIdx.x; r < a.rows_cap;
+         r += (int64_t)nblk * kMetaThreads)
+        a.recv_src[r] = -1;
+}
+
+// ---- one-CTA path -------------------------------------------------------------
+// Shared memory: cnt[E], off[E+1], cursor[E], wcnt[kMetaWarps*E].
+__global__ void __launch_bounds__(kMetaThreads) meta_single_block(MetaArgs a)
+{
+    extern __shared__ int32_t sm[];
+    int32_t *cnt = sm, *off = sm + a.E, *cursor = off + a.E + 1, *wcnt = cursor + a.E;
+    for (int32_t e = threadIdx.x; e < a.E; e += kMetaThreads)
+        cnt[e] = 0;
+    for (int32_t i = threadIdx.x; i < kMetaWarps * a.E; i += kMetaThreads)
+        wcnt[i] = 0;
+    __syncthreads();
+    block_count(a, 0, a.S, cnt);
+    __syncthreads();
+    block_offsets(cnt, off, a.E, a.pad128);
+    for (int32_t e = threadIdx.x; e < a.E; e += kMetaThreads) {
+        cursor[e] = off[e];
+        a.expert_count[e] = cnt[e];
+        a.expert_offset[e] = off[e];
+    }
+    if (threadIdx.x == 0)
+        a.expert_offset[a.E] = off[a.E];
+    for (int32_t r = threadIdx.x; r <= a.R; r += kMetaThreads)
+        a.rank_offset[r] = off[(int64_t)r * (a.E / a.R)];
+    __syncthreads();
+    block_assign(a, 0, a.S, cursor, wcnt);
+    block_fill_unused(a, cnt, off, 0, 1);
+}
+
+// ---- tiled path ----------------------------------------------------------------
+// (1) tile_hist[tile][e] = entries of tile `tile` routed to e.
+__global__ void __launch_bounds__(kMetaThreads) meta_tile_count(MetaArgs a, int32_t *tile_hist)
+{
+    extern __shared__ int32_t hist[];
+    for (int32_t e = threadIdx.x; e < a.E; e += kMetaThreads)
+        hist[e] = 0;
+    __syncthreads();
+    int64_t begin = (int64_t)blockIdx.x * kTileEntries;
+    int64_t end = begin + kTileEntries < a.S ? begin + kTileEntries : a.S;
+    block_count(a, begin, end, hist);
+    __syncthreads();
+    for (int32_t e = threadIdx.x; e < a.E; e += kMetaThreads)
+        tile_hist[(int64_t)blockIdx.x * a.E + e] = hist[e];
+}
+
+// (2) One CTA: tile_hist becomes the exclusive prefix over tiles (per expert),
+// and the counts, offsets and rank offsets are written.
+__global__ void __launch_bounds__(kMetaThreads) meta_tile_scan(MetaArgs a, int32_t *tile_hist,
+                                                               int32_t ntiles)
+{
+    extern __shared__ int32_t sm[];
+    int32_t *cnt = sm, *off = sm + a.E;
+    for (int32_t e = threadIdx.x; e < a.E; e += kMetaThreads) {
+        int32_t run = 0;
+        for (int32_t t = 0; t < ntiles; ++t) {
+            int32_t c = tile_hist[(int64_t)t * a.E + e];
+            tile_hist[(int64_t)t * a.E + e] = run;
+            run += c;
+        }
+        cnt[e] = run;
+    }
+    __syncthreads();
+    block_offsets(cnt, off, a.E, a.pad128);
+    for (int32_t e = threadIdx.x; e < a.E; e += kMetaThreads) {
+        a.expert_count[e] = cnt[e];
+        a.expert_offset[e] = off[e];
+    }
+    if (threadIdx.x == 0)
+        a.expert_offset[a.E] = off[a.E];
+    for (int32_t r = threadIdx.x; r <= a.R; r += kMetaThreads)
+        a.rank_offset[r] = off[(int64_t)r * (a.E / a.R)];
+}
+
+// (3) Slots of one tile, from offset[e] + the tile's prefix; also clears the
+// unused rows' recv_src (split over all CTAs).
+// Shared memory: cursor[E], wcnt[kMetaWarps*E].
+__global__ void __launch_bounds__(kMetaThreads) meta_tile_assign(MetaArgs a,
+                                                                 const int32_t *tile_prefix)
+{
+    extern __shared__ int32_t sm[];
+    int32_t *cursor = sm, *wcnt = sm + a.E;
+    for (int32_t e = threadIdx.x; e < a.E; e += kMetaThreads)
+        cursor[e] = a.expert_offset[e] + tile_prefix[(int64_t)blockIdx.x * a.E + e];
+    for (int32_t i = threadIdx.x; i < kMetaWarps * a.E; i += kMetaThreads)
+        wcnt[i] = 0;
+    __syncthreads();
+    int64_t begin = (int64_t)blockIdx.x * kTileEntries;
+    int64_t end = begin + kTileEntries < a.S ? begin + kTileEntries : a.S;
+    block_assign(a, begin, end, cursor, wcnt);
+    block_fill_unused(a, a.expert_count, a.expert_offset, blockIdx.x, gridDim.x);
+}
+
+inline size_t meta_single_smem(int32_t E) { return sizeof(int32_t) * ((size_t)3 * E + 1 + (size_t)kMetaWarps * E); }
+inline size_t meta_count_smem(int32_t E) { return sizeof(int32_t) * (size_t)E; }
+inline size_t meta_scan_smem(int32_t E) { return sizeof(int32_t) * ((size_t)2 * E + 1); }
+inline size_t meta_assign_smem(int32_t E) { return sizeof(int32_t) * ((size_t)E + (size_t)kMetaWarps * E); }
+
+inline int64_t meta_tiles(int64_t S) { return (S + kTileEntries - 1) / kTileEntries; }
+
+} // namespace moe

@@ -1,0 +1,304 @@
+// C ABI of the MoE dispatch / combine library: host-side validation and
+// launches.  The declarations and their contracts are in
+// include/moe_dispatch_combine.h.
+#include <cstdint>
+#include <cstring>
+
+#include <cuda_runtime.h>
+
+#include "moe_dispatch_combine.h"
+
+#include "combine.cuh"
+#include "common.cuh"
+#include "meta.cuh"
+#include "scatter.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kVersion = 100; // 0.1.0
+
+// Per-device launch facts, read once per device.
+struct DeviceInfo {
+    bool ready = false;
+    int sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+int device_info(DeviceInfo **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return MOE_ERR_CUDA;
+    DeviceInfo &d = g_dev[dev];
+    if (!d.ready) {
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        const size_t big = meta_single_smem(MOE_MAX_EXPERTS);
+        if (cudaFuncSetAttribute(meta_single_block, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)big) != cudaSuccess ||
+            cudaFuncSetAttribute(meta_tile_assign, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)meta_assign_smem(MOE_MAX_EXPERTS)) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        d.ready = true;
+    }
+    *out = &d;
+    return MOE_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_config(const moe_config *c)
+{
+    if (c == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (c->H <= 0 || c->k <= 0 || c->E <= 0 || c->R <= 0 || c->E % c->R != 0)
+        return MOE_ERR_INVALID_ARG;
+    if ((c->flags & ~(MOE_FP8 | MOE_PAD128)) != 0)
+        return MOE_ERR_INVALID_ARG;
+    if (c->H % 8 != 0 || c->E > MOE_MAX_EXPERTS || c->k > MOE_MAX_TOPK)
+        return MOE_ERR_UNSUPPORTED;
+    if ((c->flags & MOE_FP8) && c->H % 128 != 0)
+        return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+int64_t rows_capacity(const moe_config *c, int32_t T)
+{
+    const int64_t S = (int64_t)T * c->k;
+    if (!(c->flags & MOE_PAD128))
+        return S;
+    // At most min(E, S) non-empty experts, each adding at most 127 pad rows;
+    // the total is a whole number of 128-row blocks, and the bound
+    // floor((S + 127*m) / 128) blocks is reached with m-1 single-entry experts.
+    const int64_t m = S < c->E ? S : c->E;
+    return (S + 127 * m) / 128 * 128;
+}
+
+bool use_single_block(int64_t S) { return S <= kSingleBlockEntries; }
+
+size_t workspace_bytes(const moe_config *c, int32_t T)
+{
+    const int64_t S = (int64_t)T * c->k;
+    if (use_single_block(S))
+        return 0;
+    const size_t raw = (size_t)meta_tiles(S) * (size_t)c->E * sizeof(int32_t);
+    return (raw + 255) / 256 * 256;
+}
+
+int launched(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// Grid for `units` work units of a 128-thread kernel: enough CTAs to fill every
+// SM at full occupancy, fewer if there are fewer units.
+unsigned grid_for(int64_t units, int sms, int ctas_per_sm)
+{
+    int64_t cap = (int64_t)sms * ctas_per_sm;
+    int64_t g = units < cap ? units : cap;
+    return (unsigned)(g > 0 ? g : 1);
+}
+
+} // namespace
+} // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int moe_version(void) { return kVersion; }
+
+const char *moe_status_string(int status)
+{
+    switch (status) {
+    case MOE_OK:
+        return "ok";
+    case MOE_ERR_INVALID_ARG:
+        return "invalid argument";
+    case MOE_ERR_UNSUPPORTED:
+        return "unsupported configuration";
+    case MOE_ERR_CUDA:
+        return "CUDA error";
+    case MOE_ERR_DEVICE:
+        return "device reported an error";
+    default:
+        return "unknown status";
+    }
+}
+
+int64_t moe_rows_capacity(const moe_config *cfg, int32_t T)
+{
+    if (check_config(cfg) != MOE_OK || T < 0)
+        return -1;
+    return rows_capacity(cfg, T);
+}
+
+size_t moe_workspace_bytes(const moe_config *cfg, int32_t T)
+{
+    if (check_config(cfg) != MOE_OK || T < 0)
+        return 0;
+    return workspace_bytes(cfg, T);
+}
+
+int moe_dispatch_sizes_for(const moe_config *cfg, int32_t T, int64_t rows_cap,
+                           moe_dispatch_sizes *sizes)
+{
+    int st = check_config(cfg);
+    if (st != MOE_OK)
+        return st;
+    if (sizes == nullptr || T < 0 || rows_cap < 0)
+        return MOE_ERR_INVALID_ARG;
+    const bool fp8 = cfg->flags & MOE_FP8;
+    sizes->recv_x = (size_t)rows_cap * cfg->H * (fp8 ? 1 : 2);
+    sizes->recv_scale = fp8 ? (size_t)rows_cap * (cfg->H / 128) * sizeof(float) : 0;
+    sizes->expert_count = (size_t)cfg->E * sizeof(int32_t);
+    sizes->expert_offset = (size_t)(cfg->E + 1) * sizeof(int32_t);
+    sizes->rank_offset = (size_t)(cfg->R + 1) * sizeof(int32_t);
+    sizes->recv_src = (size_t)rows_cap * sizeof(int32_t);
+    sizes->slot = (size_t)T * cfg->k * sizeof(int32_t);
+    return MOE_OK;
+}
+
+int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t *topk_idx,
+                 const float *topk_w, const moe_dispatch_out *out, int32_t *slot,
+                 void *workspace, size_t workspace_bytes_given, int32_t *dev_err, void *stream,
+                 moe_handle *handle)
+{
+    int st = check_config(cfg);
+    if (st != MOE_OK)
+        return st;
+    if (T < 0 || out == nullptr || handle == nullptr || dev_err == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    const bool fp8 = cfg->flags & MOE_FP8;
+    const int64_t S = (int64_t)T * cfg->k;
+    const int64_t rows_cap = out->rows_cap;
+    if (rows_cap < 0 || rows_cap > INT32_MAX || S > INT32_MAX)
+        return MOE_ERR_INVALID_ARG;
+    if (rows_capacity(cfg, T) > INT32_MAX)
+        return MOE_ERR_UNSUPPORTED;
+    if (out->expert_count == nullptr || out->expert_offset == nullptr ||
+        out->rank_offset == nullptr || (rows_cap > 0 && out->recv_src == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (x == nullptr || topk_idx == nullptr || topk_w == nullptr || slot == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    if (rows_cap > 0 && (out->recv_x == nullptr || (fp8 && out->recv_scale == nullptr)))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(out->recv_x) || (fp8 && !aligned16(out->recv_scale)))
+        return MOE_ERR_INVALID_ARG;
+    const size_t need_ws = workspace_bytes(cfg, T);
+    if (need_ws > 0 && (workspace == nullptr || workspace_bytes_given < need_ws))
+        return MOE_ERR_INVALID_ARG;
+
+    DeviceInfo *dev = nullptr;
+    if ((st = device_info(&dev)) != MOE_OK)
+        return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    MetaArgs m;
+    m.topk_idx = topk_idx;
+    m.S = S;
+    m.k = cfg->k;
+    m.E = cfg->E;
+    m.R = cfg->R;
+    m.pad128 = (cfg->flags & MOE_PAD128) ? 1 : 0;
+    m.rows_cap = rows_cap;
+    m.expert_count = out->expert_count;
+    m.expert_offset = out->expert_offset;
+    m.rank_offset = out->rank_offset;
+    m.slot = slot;
+    m.recv_src = out->recv_src;
+    m.err = dev_err;
+
+    if (use_single_block(S)) {
+        meta_single_block<<<1, kMetaThreads, meta_single_smem(cfg->E), s>>>(m);
+        if ((st = launched(cudaGetLastError())) != MOE_OK)
+            return st;
+    } else {
+        const int64_t ntiles = meta_tiles(S);
+        int32_t *tile_hist = static_cast<int32_t *>(workspace);
+        meta_tile_count<<<(unsigned)ntiles, kMetaThreads, meta_count_smem(cfg->E), s>>>(m, tile_hist);
+        meta_tile_scan<<<1, kMetaThreads, meta_scan_smem(cfg->E), s>>>(m, tile_hist, (int32_t)ntiles);
+        meta_tile_assign<<<(unsigned)ntiles, kMetaThreads, meta_assign_smem(cfg->E), s>>>(m, tile_hist);
+        if ((st = launched(cudaGetLastError())) != MOE_OK)
+            return st;
+    }
+
+    if (T > 0) {
+        ScatterArgs a;
+        a.x = static_cast<const uint16_t *>(x);
+        a.slot = slot;
+        a.T = T;
+        a.H = cfg->H;
+        a.k = cfg->k;
+        a.parts = (cfg->H / 8 + kScatterThreads - 1) / kScatterThreads;
+        a.recv_x = out->recv_x;
+        a.recv_scale = out->recv_scale;
+        const unsigned grid = grid_for((int64_t)T * a.parts, dev->sms, 16);
+        if (fp8)
+            scatter_rows<true><<<grid, kScatterThreads, 0, s>>>(a);
+        else
+            scatter_rows<false><<<grid, kScatterThreads, 0, s>>>(a);
+        if ((st = launched(cudaGetLastError())) != MOE_OK)
+            return st;
+    }
+
+    handle->cfg = *cfg;
+    handle->T = T;
+    handle->slot = slot;
+    handle->topk_w = topk_w;
+    handle->rows_cap = rows_cap;
+    return MOE_OK;
+}
+
+int moe_combine(const moe_handle *handle, const void *expert_out, void *y, int32_t *dev_err,
+                void *stream)
+{
+    if (handle == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    int st = check_config(&handle->cfg);
+    if (st != MOE_OK)
+        return st;
+    const moe_config &c = handle->cfg;
+    if (handle->T < 0 || handle->rows_cap < 0)
+        return MOE_ERR_INVALID_ARG;
+    if (handle->T == 0)
+        return MOE_OK;
+    if (handle->slot == nullptr || handle->topk_w == nullptr || y == nullptr ||
+        (handle->rows_cap > 0 && expert_out == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(expert_out) || !aligned16(y))
+        return MOE_ERR_INVALID_ARG;
+    DeviceInfo *dev = nullptr;
+    if ((st = device_info(&dev)) != MOE_OK)
+        return st;
+    CombineArgs a;
+    a.expert_out = static_cast<const uint16_t *>(expert_out);
+    a.slot = handle->slot;
+    a.w = handle->topk_w;
+    a.T = handle->T;
+    a.H = c.H;
+    a.k = c.k;
+    a.parts = (c.H / 8 + kCombineThreads - 1) / kCombineThreads;
+    a.rows_cap = handle->rows_cap;
+    a.y = static_cast<uint16_t *>(y);
+    a.err = dev_err;
+    const unsigned grid = grid_for((int64_t)a.T * a.parts, dev->sms, 16);
+    combine_rows<<<grid, kCombineThreads, 0, static_cast<cudaStream_t>(stream)>>>(a);
+    return launched(cudaGetLastError());
+}
+
+int moe_check(int32_t *dev_err, void *stream, int32_t *bits_out)
+{
+    if (dev_err == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t bits = 0;
+    if (cudaMemcpyAsync(&bits, dev_err, sizeof bits, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess ||
+        cudaMemsetAsync(dev_err, 0, sizeof(int32_t), s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (bits_out != nullptr)
+        *bits_out = bits;
+    return bits ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+} // extern "C"

@@ -1,0 +1,218 @@
+/*
+ * moe_dispatch_combine.h -- C ABI of the B200 MoE token dispatch / combine library.
+ *
+ * What the calls compute
+ * ----------------------
+ * "Enabling trillion-parameter models on AWS EFA", section "Introdução" and
+ * section "MoE all-to-all sobre EFA": a dispatch step takes the tokens and the
+ * experts chosen for each token and sends each token to where its experts live;
+ * its dual, combine, takes the experts' processed rows back and forms each
+ * token's routing-weighted sum.  Section "Buffers de Envio e Recebimento" and
+ * section "Despacho e Combinação" of the same page fix the layout: tokens are
+ * counted per expert, the cumulative sum of the counts gives each expert's
+ * offset, and each expert's tokens are packed contiguously from there.  Section
+ * "Avaliação" evaluates the dispatch with block-scaled fp8 payloads and the
+ * combine in bf16; "Lower latency and higher throughput with multi-node
+ * DeepSeek deployment", section "Quantização", defines the blocks: one scale
+ * per 128-element activation vector.
+ *
+ * On one GPU the "ranks" that host experts are virtual: rank r owns experts
+ * [r*E/R, (r+1)*E/R) (the expert-parallel split of the DeepSeek page, section
+ * "Paralelismo de Especialistas"), and its receive buffer is the contiguous row
+ * range [rank_offset[r], rank_offset[r+1]) of one allocation.
+ *
+ * Conventions
+ * -----------
+ * - Every pointer argument except `cfg`, `out`, `handle`, `bits_out` and
+ *   `sizes` is a DEVICE pointer.  The caller allocates and owns every buffer;
+ *   the library allocates nothing and frees nothing.
+ * - All arrays are dense and row-major.  bf16 data is passed as 16-bit IEEE
+ *   bfloat16 bit patterns; fp8 data as OCP e4m3 ("e4m3fn") bytes.
+ * - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every call
+ *   only enqueues work on it and returns; nothing waits for the GPU except
+ *   moe_check.  No call reads data back to the host, so a dispatch/combine
+ *   sequence can be captured in a CUDA graph.
+ * - Host-side argument errors return a negative status and enqueue nothing.
+ * - Device-side errors (an expert id outside [0,E), a receive row at or past
+ *   the capacity) never trap: the offending entry is dropped (its slot is -1
+ *   and nothing is stored for it) and a bit is OR-ed into the caller's device
+ *   error word.  moe_check reads and clears that word.
+ */
+#ifndef MOE_DISPATCH_COMBINE_H
+#define MOE_DISPATCH_COMBINE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+/* Entry points are exported from the shared library; everything else is hidden. */
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* moe_config.flags */
+#define MOE_FP8 1    /* payload as e4m3 codes plus one fp32 scale per 128 columns */
+#define MOE_PAD128 2 /* every expert segment padded to a multiple of 128 rows      */
+
+/* Host status codes. */
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG -1 /* a null or misaligned pointer, a bad size        */
+#define MOE_ERR_UNSUPPORTED -2 /* a valid request outside what the kernels cover */
+#define MOE_ERR_CUDA -3        /* a CUDA runtime call or launch failed            */
+#define MOE_ERR_DEVICE -4      /* moe_check: the device error word was non-zero  */
+
+/* Bits of the device error word. */
+#define MOE_DEV_BAD_INDEX 1 /* dispatch: an expert id outside [0, E)                  */
+#define MOE_DEV_CAPACITY 2  /* dispatch: a receive row at or past rows_cap            */
+#define MOE_DEV_TIMEOUT 4   /* a bounded device wait gave up                          */
+#define MOE_DEV_BAD_SLOT 8  /* combine: a slot outside [-1, rows_cap) in the handle   */
+
+/* Limits of this build. */
+#define MOE_MAX_EXPERTS 2048 /* E */
+#define MOE_MAX_TOPK 64      /* k */
+
+/*
+ * Problem description.
+ *   H      hidden size; a multiple of 8 (16-byte rows), and of 128 with MOE_FP8.
+ *   k      experts per token, 1..MOE_MAX_TOPK.
+ *   E      experts, 1..MOE_MAX_EXPERTS.
+ *   R      virtual ranks; E must be a multiple of R.
+ *   flags  OR of MOE_FP8, MOE_PAD128.
+ */
+typedef struct {
+    int32_t H, k, E, R, flags;
+} moe_config;
+
+/*
+ * Caller-allocated dispatch outputs (device pointers).
+ *   recv_x        [rows_cap, H] bf16, or [rows_cap, H] e4m3 bytes with MOE_FP8.
+ *                 Row slot[t,j] holds token t's payload; 16-byte aligned.
+ *   recv_scale    [rows_cap, H/128] fp32 with MOE_FP8 (16-byte aligned), else NULL.
+ *   expert_count  [E]     tokens routed to each expert.
+ *   expert_offset [E+1]   first row of each expert's segment; expert_offset[E]
+ *                         is the number of rows in use.
+ *   rank_offset   [R+1]   rank_offset[r] = expert_offset[r*E/R].
+ *   recv_src      [rows_cap] the routing entry t*k+j a row holds, -1 for a row
+ *                 that holds none (padding and unused capacity).
+ *   rows_cap      rows of recv_x / recv_scale / recv_src.  moe_rows_capacity
+ *                 gives the worst case; a smaller capacity is allowed, and
+ *                 entries that do not fit are dropped with MOE_DEV_CAPACITY.
+ * Rows without an entry are not written in recv_x and recv_scale.
+ */
+typedef struct {
+    void *recv_x;
+    float *recv_scale;
+    int32_t *expert_count;
+    int32_t *expert_offset;
+    int32_t *rank_offset;
+    int32_t *recv_src;
+    int64_t rows_cap;
+} moe_dispatch_out;
+
+/*
+ * What combine needs from a dispatch ("Buffers de Envio e Recebimento": the
+ * combine already has the routing information from the dispatch phase).
+ * Filled by moe_dispatch; plain data, copyable, valid while the buffers it
+ * points to live.
+ *   slot    [T, k] int32 device: receive row of entry (t, j), or -1 if dropped.
+ *   topk_w  [T, k] fp32 device: the routing weights passed to moe_dispatch.
+ */
+typedef struct {
+    moe_config cfg;
+    int32_t T;
+    int32_t *slot;
+    const float *topk_w;
+    int64_t rows_cap;
+} moe_handle;
+
+/* Byte sizes of the dispatch buffers for a given capacity (host-only helper). */
+typedef struct {
+    size_t recv_x, recv_scale, expert_count, expert_offset, rank_offset, recv_src, slot;
+} moe_dispatch_sizes;
+
+/*
+ * Worst-case receive rows for T tokens: T*k; with MOE_PAD128 the most 128-row
+ * blocks T*k entries can fill over min(E, T*k) experts, times 128.
+ * Returns -1 for an invalid cfg or T < 0.
+ */
+MOE_API int64_t moe_rows_capacity(const moe_config *cfg, int32_t T);
+
+/* Fills *sizes for T tokens and rows_cap rows; returns a status. */
+MOE_API int moe_dispatch_sizes_for(const moe_config *cfg, int32_t T, int64_t rows_cap,
+                           moe_dispatch_sizes *sizes);
+
+/*
+ * Bytes of device scratch moe_dispatch needs for T tokens (0 for small
+ * batches).  Returns 0 and sets nothing for an invalid cfg.
+ */
+MOE_API size_t moe_workspace_bytes(const moe_config *cfg, int32_t T);
+
+/*
+ * Dispatch T tokens (section "Despacho e Combinação" of the EFA page: per-expert
+ * counts, their cumulative sum as offsets, tokens packed contiguously per
+ * expert).
+ *
+ *   x         [T, H] bf16, 16-byte aligned.
+ *   topk_idx  [T, k] int32 expert ids.
+ *   topk_w    [T, k] fp32 routing weights; not read here, only recorded in the
+ *             handle for moe_combine (must stay alive until then).
+ *   out       caller-allocated outputs, see moe_dispatch_out.
+ *   slot      [T, k] int32 output: receive row of each entry, -1 if dropped.
+ *   workspace device scratch of at least moe_workspace_bytes(cfg, T) bytes
+ *             (may be NULL when that is 0).  Its contents are not preserved.
+ *   dev_err   device int32 error word; bits are OR-ed in, never cleared here.
+ *   handle    host struct filled on success.
+ *
+ * Inside each expert's segment, entries are in (token, k) order, so the result
+ * is unique and deterministic.  With MOE_FP8 each 128-column block of a token
+ * gets scale = amax/448 and codes e4m3(x/scale) (both divisions IEEE binary32
+ * round-to-nearest; codes rounded to nearest-even and saturated to +-448; an
+ * all-zero block gets scale 0 and codes 0), and every slot of the token gets
+ * the same codes and scales.
+ * Returns MOE_OK or a negative status (nothing enqueued on error).
+ */
+MOE_API int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t *topk_idx,
+                 const float *topk_w, const moe_dispatch_out *out, int32_t *slot,
+                 void *workspace, size_t workspace_bytes, int32_t *dev_err, void *stream,
+                 moe_handle *handle);
+
+/*
+ * Combine (EFA page, sections "Introdução" and "Despacho e Combinação"; DeepSeek
+ * page, section "Paralelismo de Especialistas"): for every token t,
+ *   y[t, :] = bf16( sum_{j=0..k-1} topk_w[t,j] * expert_out[slot[t,j], :] )
+ * accumulated in fp32 with one fused multiply-add per j in ascending j,
+ * starting from 0, then rounded to nearest-even bf16.  Entries with slot -1
+ * are skipped.  The weights are used as given (no division by their sum).
+ *
+ *   handle      from moe_dispatch.
+ *   expert_out  [rows_cap, H] bf16 in the receive layout, 16-byte aligned.
+ *   y           [T, H] bf16 output, 16-byte aligned.
+ *   dev_err     device error word (may be NULL): MOE_DEV_BAD_SLOT.
+ * Returns MOE_OK or a negative status.
+ */
+MOE_API int moe_combine(const moe_handle *handle, const void *expert_out, void *y, int32_t *dev_err,
+                void *stream);
+
+/*
+ * Waits for `stream`, reads the device error word, clears it (stream-ordered),
+ * and stores it in *bits_out when not NULL.  Returns MOE_OK if it was 0,
+ * MOE_ERR_DEVICE if not, MOE_ERR_CUDA if the stream failed.
+ */
+MOE_API int moe_check(int32_t *dev_err, void *stream, int32_t *bits_out);
+
+/* Short English text for a status code. */
+MOE_API const char *moe_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+MOE_API int moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_DISPATCH_COMBINE_H */

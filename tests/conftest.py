@@ -18,3 +18,9 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_sessionstart(session):
+    # The library is built in place (nvcc cross-compiles; no GPU needed).
+    from tests._lib import ensure_built
+    ensure_built()

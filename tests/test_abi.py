@@ -1,0 +1,112 @@
+"""The C ABI without a GPU: the library loads, exports what the header declares,
+and its host-only calls (sizing, argument validation) behave as documented."""
+import ctypes
+import re
+
+import pytest
+
+import oracle
+from tests._lib import HEADER
+
+import combine_route_meta_b200 as moe
+
+
+def _declared():
+    text = open(HEADER).read()
+    return re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text)
+
+
+def test_header_declares_the_entry_points():
+    names = set(_declared())
+    for n in ["moe_dispatch", "moe_combine", "moe_rows_capacity", "moe_workspace_bytes",
+              "moe_dispatch_sizes_for", "moe_check", "moe_status_string", "moe_version"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(moe.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_binding_mirrors_c_names():
+    for name in _declared():
+        assert callable(getattr(moe, name)), name
+
+
+def test_version_and_status_strings():
+    assert moe.moe_version() >= 100
+    assert moe.moe_status_string(moe.OK) == b"ok"
+    assert moe.moe_status_string(moe.ERR_UNSUPPORTED) == b"unsupported configuration"
+
+
+@pytest.mark.parametrize("T,k,E,pad", [(0, 8, 256, True), (1, 1, 4, True), (16, 2, 8, False),
+                                       (128, 8, 256, False), (256, 8, 256, True),
+                                       (1024, 8, 256, True), (16384, 8, 256, True),
+                                       (3, 2, 1, True), (7, 3, 1000, True)])
+def test_rows_capacity_matches_oracle(T, k, E, pad):
+    cfg = moe.make_config(128, k, E, 1, fp8=False, pad128=pad)
+    assert moe.rows_capacity(cfg, T) == oracle.rows_capacity(T, k, E, pad)
+
+
+def test_config_validation_statuses():
+    bad = [
+        (moe.make_config(0, 8, 256, 8, False), moe.ERR_INVALID_ARG),
+        (moe.make_config(7168, 0, 256, 8, False), moe.ERR_INVALID_ARG),
+        (moe.make_config(7168, 8, 256, 7, False), moe.ERR_INVALID_ARG),   # E % R
+        (moe.make_config(7168, 8, 0, 1, False), moe.ERR_INVALID_ARG),
+        (moe.make_config(100, 8, 256, 8, False), moe.ERR_UNSUPPORTED),    # H % 8
+        (moe.make_config(7176, 8, 256, 8, True), moe.ERR_UNSUPPORTED),    # fp8 needs H % 128
+        (moe.make_config(128, 8, 4096, 8, False), moe.ERR_UNSUPPORTED),   # E > max
+        (moe.make_config(128, 65, 256, 8, False), moe.ERR_UNSUPPORTED),   # k > max
+    ]
+    for cfg, want in bad:
+        sizes = moe.moe_dispatch_sizes()
+        assert moe.moe_dispatch_sizes_for(ctypes.byref(cfg), 4, 32, ctypes.byref(sizes)) == want
+        assert moe.moe_rows_capacity(ctypes.byref(cfg), 4) == -1
+    cfg = moe.moe_config(128, 2, 8, 2, 4)  # unknown flag bit
+    assert moe.moe_rows_capacity(ctypes.byref(cfg), 4) == -1
+
+
+def test_dispatch_rejects_bad_arguments_before_touching_the_gpu():
+    cfg = moe.make_config(256, 2, 8, 2, fp8=False)
+    out = moe.moe_dispatch_out(16, None, 16, 16, 16, 16, 32)
+    h = moe.moe_handle()
+    P = ctypes.c_void_p
+    # null error word
+    assert moe.moe_dispatch(ctypes.byref(cfg), 16, P(16), P(16), P(16), ctypes.byref(out), P(16),
+                            None, 0, None, None, ctypes.byref(h)) == moe.ERR_INVALID_ARG
+    # misaligned x
+    assert moe.moe_dispatch(ctypes.byref(cfg), 16, P(18), P(16), P(16), ctypes.byref(out), P(16),
+                            None, 0, P(16), None, ctypes.byref(h)) == moe.ERR_INVALID_ARG
+    # negative T
+    assert moe.moe_dispatch(ctypes.byref(cfg), -1, P(16), P(16), P(16), ctypes.byref(out), P(16),
+                            None, 0, P(16), None, ctypes.byref(h)) == moe.ERR_INVALID_ARG
+    # missing workspace for a batch that needs one
+    big = moe.make_config(256, 8, 8, 2, fp8=False)
+    assert moe.workspace_bytes(big, 4096) > 0
+    out2 = moe.moe_dispatch_out(16, None, 16, 16, 16, 16, 4096 * 8)
+    assert moe.moe_dispatch(ctypes.byref(big), 4096, P(16), P(16), P(16), ctypes.byref(out2), P(16),
+                            None, 0, P(16), None, ctypes.byref(h)) == moe.ERR_INVALID_ARG
+    # fp8 without a scale buffer
+    f8 = moe.make_config(256, 2, 8, 2, fp8=True)
+    assert moe.moe_dispatch(ctypes.byref(f8), 16, P(16), P(16), P(16), ctypes.byref(out), P(16),
+                            None, 0, P(16), None, ctypes.byref(h)) == moe.ERR_INVALID_ARG
+
+
+def test_combine_rejects_bad_arguments():
+    h = moe.moe_handle(moe.make_config(256, 2, 8, 2, False), 16, 16, 16, 32)
+    P = ctypes.c_void_p
+    assert moe.moe_combine(None, P(16), P(16), None, None) == moe.ERR_INVALID_ARG
+    assert moe.moe_combine(ctypes.byref(h), P(16), None, None, None) == moe.ERR_INVALID_ARG
+    assert moe.moe_combine(ctypes.byref(h), P(8), P(16), None, None) == moe.ERR_INVALID_ARG
+    h.T = 0  # nothing to do: returns without launching
+    assert moe.moe_combine(ctypes.byref(h), None, None, None, None) == moe.OK
+
+
+def test_sizes_for_fp8():
+    cfg = moe.make_config(7168, 8, 256, 8, fp8=True)
+    s = moe.moe_dispatch_sizes()
+    assert moe.moe_dispatch_sizes_for(ctypes.byref(cfg), 128, 1024, ctypes.byref(s)) == moe.OK
+    assert s.recv_x == 1024 * 7168 and s.recv_scale == 1024 * 56 * 4
+    assert s.expert_offset == 257 * 4 and s.rank_offset == 9 * 4 and s.slot == 128 * 8 * 4
