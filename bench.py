@@ -80,16 +80,22 @@ def recorded_traffic(kernel_file, workload):
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    """nvidia-smi samples of SM clock and throttle reasons around the timed region.
+
+    Samples arrive every 100 ms; those inside the timed window are used, and if the
+    window is shorter than the sampling period, the nearest sample on each side.
+    """
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.lines = []
+        self.samples = []  # (monotonic time, sm_mhz, max_mhz, active reasons)
+        self.t0 = self.t1 = None
 
     def start(self):
         try:
@@ -104,7 +110,30 @@ class ClockSampler:
 
     def _read(self):
         for ln in self.proc.stdout:
-            self.lines.append(ln.strip())
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz, mx = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            act = [n for n, v in zip(self.REASONS, parts[5:9]) if v.lower().startswith("active")]
+            self.samples.append((time.monotonic(), mhz, mx, act))
+
+    def count(self):
+        return len(self.samples) if self.proc is not None else 10**9
+
+    def mark_start(self):
+        self.t0 = time.monotonic()
+
+    def mark_end(self):
+        self.t1 = time.monotonic()
+        if self.proc is not None:
+            deadline = time.monotonic() + 1.0
+            n = len([s for s in self.samples if s[0] > self.t1])
+            while n == 0 and time.monotonic() < deadline:
+                time.sleep(0.02)
+                n = len([s for s in self.samples if s[0] > self.t1])
 
     def stop(self):
         if self.proc is None:
@@ -115,24 +144,18 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.t.join(timeout=2)
-        mhz, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                mhz.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not mhz:
+        inside = [s for s in self.samples if self.t0 <= s[0] <= self.t1]
+        window = "inside"
+        if not inside:
+            window = "adjacent"
+            before = [s for s in self.samples if s[0] < self.t0][-1:]
+            after = [s for s in self.samples if s[0] > self.t1][:1]
+            inside = before + after
+        if not inside:
             return None
-        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(mhz)}
+        reasons = sorted({r for s in inside for r in s[3]})
+        return {"sm_mhz": statistics.median(s[1] for s in inside), "sm_max_mhz": inside[-1][2],
+                "reasons": reasons, "samples": len(inside), "window": window}
 
 
 # ---- CPU oracle arm ---------------------------------------------------------------
@@ -208,8 +231,12 @@ def run_gpu(args, rank, world):
         raise SystemExit("identity experts need a bf16 dispatch")
     y = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev)
 
+    # L2 flush between steps: write a 2x-L2 buffer, then read another 2x-L2 buffer,
+    # so the step starts with no payload lines cached and no dirty lines to evict.
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    flush_w = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    flush_r = torch.zeros(2 * l2 // 4, dtype=torch.int32, device=dev)
+    flush_sink = torch.empty((), dtype=torch.int64, device=dev)
     stream = torch.cuda.Stream(device=dev)
 
     def do_dispatch():
@@ -236,7 +263,8 @@ def run_gpu(args, rank, world):
 
     def step(evs):
         with torch.cuda.stream(stream):
-            flush.zero_()
+            flush_w.zero_()
+            torch.sum(flush_r, dim=0, dtype=torch.int64, out=flush_sink)
             torch.cuda._sleep(20_000)  # lets the host queue the step before the GPU reaches it
             evs[0].record(stream)
             g_disp.replay()
@@ -244,8 +272,17 @@ def run_gpu(args, rank, world):
             g_comb.replay()
             evs[2].record(stream)
 
-    for _ in range(args.warmup):
+    # Warm-up: at least W steps, and on until the clock sampler reports (the GPU
+    # is then under load when the timed region starts).
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    t_warm = time.monotonic()
+    n = 0
+    while n < args.warmup or (sampler.count() < 2 and time.monotonic() - t_warm < 5.0):
         step([torch.cuda.Event(enable_timing=True) for _ in range(3)])
+        n += 1
+        if n % 20 == 0:
+            torch.cuda.synchronize()
     torch.cuda.synchronize()
 
     dist = None
@@ -253,8 +290,7 @@ def run_gpu(args, rank, world):
         import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
-    sampler = ClockSampler(dev.index)
-    sampler.start()
+    sampler.mark_start()
     all_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     for evs in all_evs:
         step(evs)
@@ -262,6 +298,7 @@ def run_gpu(args, rank, world):
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
+    sampler.mark_end()
     clocks = sampler.stop()
 
     disp_ms = [a.elapsed_time(b) for a, b, _ in all_evs]
@@ -315,7 +352,7 @@ def run_gpu(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

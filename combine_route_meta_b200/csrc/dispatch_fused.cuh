@@ -1,0 +1,171 @@
+// Dispatch of a small batch in one launch: routing metadata and payload fused.
+//
+// Same results as the metadata kernels followed by the scatter (counts, offsets,
+// (token, k)-ordered slots, bf16 rows or e4m3 codes with per-128 scales; the
+// steps of "Enabling trillion-parameter models on AWS EFA", section "Despacho e
+// Combinação"), shaped for decode batches where one launch and one DRAM round
+// trip cost more than the bytes.
+//
+// One CTA per token t.  The CTA first issues the loads of x[t] (they do not
+// depend on the routing), then reads all S = T*k expert ids (a few KB, served
+// from L2 after the first CTA) and builds in shared memory the histogram of all
+// entries and, in the same pass, the histogram of the entries that come before
+// token t.  With the exclusive scan of the (padded) counts, the slot of (t, j)
+// with expert e is
+//   offset[e] + before_t[e] + #{j' < j : topk_idx[t, j'] == e},
+// which is the stable (token, k) order.  The CTA then stores (or quantises and
+// stores) its row to its k slots.  CTA 0 also writes the per-expert counts and
+// offsets; the padding rows' recv_src = -1 is split over all CTAs.  The
+// redundant histogram per CTA is a few hundred instructions per warp at decode
+// sizes, which is why this path is limited to S <= kFusedMaxEntries.
+#pragma once
+
+#include "common.cuh"
+#include "meta.cuh"
+#include "scatter.cuh"
+
+namespace moe {
+
+constexpr int kFusedMaxEntries = 2048;
+constexpr int kFusedMaxK = 16;
+constexpr int kFusedMaxThreads = 512;
+constexpr int kFusedMaxVpt = 4; // 16-byte vectors per thread: rows up to 2048 vectors
+
+struct FusedArgs {
+    const uint16_t *x;
+    const int32_t *topk_idx;
+    int32_t T, H, k, E, R, pad128;
+    int64_t rows_cap;
+    void *recv_x;
+    float *recv_scale;
+    int32_t *expert_count, *expert_offset, *rank_offset, *recv_src, *slot;
+    int32_t *err;
+};
+
+// Shared memory: hist[E], before[E], off[E+1].
+inline size_t fused_smem(int32_t E) { return sizeof(int32_t) * ((size_t)3 * E + 1); }
+
+template <int kVpt, bool kFp8>
+__global__ void __launch_bounds__(kFusedMaxThreads) dispatch_fused(FusedArgs a)
+{
+    extern __shared__ int32_t sm[];
+    int32_t *hist = sm, *before = sm + a.E, *off = sm + 2 * a.E;
+    __shared__ int32_t s_slot[kFusedMaxK];
+
+    const int32_t t = blockIdx.x;
+    const int nt = blockDim.x;
+    const unsigned lane = lane_id();
+    const int32_t nvec = a.H / 8;
+
+    // 1. The row's loads go out first.
+    uint4 val[kVpt];
+#pragma unroll
+    for (int i = 0; i < kVpt; ++i) {
+        const int32_t v = threadIdx.x + i * nt;
+        val[i] = v < nvec ? ld_stream_v4(a.x + (int64_t)t * a.H + (int64_t)v * 8)
+                          : make_uint4(0u, 0u, 0u, 0u);
+    }
+
+    // 2. Histograms of all entries and of the entries before token t.
+    for (int32_t e = threadIdx.x; e < a.E; e += nt) {
+        hist[e] = 0;
+        before[e] = 0;
+    }
+    __syncthreads();
+    const int64_t S = (int64_t)a.T * a.k;
+    const int64_t mine = (int64_t)t * a.k;
+    for (int64_t base = 0; base < S; base += nt) {
+        const int64_t i = base + threadIdx.x;
+        int32_t e = -1;
+        if (i < S) {
+            e = __ldg(a.topk_idx + i);
+            if (e < 0 || e >= a.E) {
+                if (t == 0)
+                    raise_error(a.err, MOE_DEV_BAD_INDEX);
+                e = -1;
+            }
+        }
+        const unsigned peers = __match_any_sync(kFullMask, e);
+        const unsigned below = __ballot_sync(kFullMask, i < mine);
+        if (e >= 0 && lane == (unsigned)(__ffs(peers) - 1)) {
+            atomicAdd(&hist[e], __popc(peers));
+            const int nb = __popc(peers & below);
+            if (nb)
+                atomicAdd(&before[e], nb);
+        }
+    }
+    __syncthreads();
+
+    // 3. Offsets (exclusive scan of the padded counts).
+    block_offsets(hist, off, a.E, a.pad128);
+
+    // 4. This token's slots.
+    if (threadIdx.x < a.k) {
+        const int j = threadIdx.x;
+        const int32_t e = __ldg(a.topk_idx + mine + j);
+        int32_t s = -1;
+        if (e >= 0 && e < a.E) {
+            int32_t dup = 0;
+            for (int jj = 0; jj < j; ++jj)
+                dup += __ldg(a.topk_idx + mine + jj) == e;
+            const int64_t row = (int64_t)off[e] + before[e] + dup;
+            if (row < a.rows_cap) {
+                s = (int32_t)row;
+                a.recv_src[row] = (int32_t)(mine + j);
+            } else {
+                raise_error(a.err, MOE_DEV_CAPACITY);
+            }
+        }
+        a.slot[mine + j] = s;
+        s_slot[j] = s;
+    }
+    if (t == 0) {
+        for (int32_t e = threadIdx.x; e < a.E; e += nt) {
+            a.expert_count[e] = hist[e];
+            a.expert_offset[e] = off[e];
+        }
+        if (threadIdx.x == 0)
+            a.expert_offset[a.E] = off[a.E];
+        for (int32_t r = threadIdx.x; r <= a.R; r += nt)
+            a.rank_offset[r] = off[(int64_t)r * (a.E / a.R)];
+    }
+    block_fill_unused(a.rows_cap, a.E, a.recv_src, hist, off, t, gridDim.x);
+    __syncthreads();
+
+    // 5. Payload to the k slots.
+    if constexpr (kFp8) {
+        uint8_t *rx = static_cast<uint8_t *>(a.recv_x);
+        const int32_t nb = a.H / 128;
+#pragma unroll
+        for (int i = 0; i < kVpt; ++i) {
+            const int32_t v = threadIdx.x + i * nt;
+            float scale;
+            const uint2 codes = quantise_vec_e4m3(val[i], scale);
+            if (v >= nvec)
+                continue;
+            for (int32_t j = 0; j < a.k; ++j) {
+                const int32_t s = s_slot[j];
+                if (s < 0)
+                    continue;
+                st_v2(rx + (int64_t)s * a.H + (int64_t)v * 8, codes);
+                if ((lane & 15) == 0)
+                    a.recv_scale[(int64_t)s * nb + v / 16] = scale;
+            }
+        }
+    } else {
+        uint16_t *rx = static_cast<uint16_t *>(a.recv_x);
+        for (int32_t j = 0; j < a.k; ++j) {
+            const int32_t s = s_slot[j];
+            if (s < 0)
+                continue;
+#pragma unroll
+            for (int i = 0; i < kVpt; ++i) {
+                const int32_t v = threadIdx.x + i * nt;
+                if (v < nvec)
+                    st_v4(rx + (int64_t)s * a.H + (int64_t)v * 8, val[i]);
+            }
+        }
+    }
+}
+
+} // namespace moe

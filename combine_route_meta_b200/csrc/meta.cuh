@@ -81,16 +81,18 @@ __device__ __forceinline__ void block_count(const MetaArgs &a, int64_t begin, in
 
 // Exclusive scan of the (optionally 128-padded) counts in shared memory:
 // off[e] = sum_{e' < e} seg(e'), off[E] = total.  `cnt` and `off` may not alias.
-// Uses the whole block; ends with a barrier.
+// Any block size that is a multiple of 32 (up to 1024); uses the whole block
+// and ends with a barrier.
 __device__ void block_offsets(const int32_t *cnt, int32_t *off, int32_t E, int32_t pad128)
 {
-    __shared__ int32_t warp_sums[kMetaWarps];
+    __shared__ int32_t warp_sums[32];
     __shared__ int32_t carry;
     if (threadIdx.x == 0)
         carry = 0;
     __syncthreads();
     const unsigned lane = lane_id(), warp = threadIdx.x / kWarp;
-    for (int32_t base = 0; base < E; base += kMetaThreads) {
+    const int nt = blockDim.x;
+    for (int32_t base = 0; base < E; base += nt) {
         int32_t e = base + threadIdx.x;
         int32_t v = 0;
         if (e < E) {
@@ -114,7 +116,7 @@ __device__ void block_offsets(const int32_t *cnt, int32_t *off, int32_t E, int32
         if (e < E)
             off[e] = before + incl - v;
         __syncthreads();
-        if (threadIdx.x == kMetaThreads - 1)
+        if (threadIdx.x == nt - 1)
             carry = before + incl;
         __syncthreads();
     }
@@ -171,19 +173,23 @@ __device__ __forceinline__ void block_assign(const MetaArgs &a, int64_t begin, i
 }
 
 // recv_src = -1 on rows that hold no entry: each expert's padding, and the rows
-// from expert_offset[E] to rows_cap.  Work is split over `nblk` blocks.
-__device__ __forceinline__ void block_fill_unused(const MetaArgs &a, const int32_t *cnt,
-                                                  const int32_t *off, int blk, int nblk)
+// from expert_offset[E] to rows_cap.  Work is split over `nblk` blocks; inside
+// a block, one warp clears one expert's padding (at most 127 rows).
+__device__ __forceinline__ void block_fill_unused(int64_t rows_cap, int32_t E, int32_t *recv_src,
+                                                  const int32_t *cnt, const int32_t *off, int blk,
+                                                  int nblk)
 {
-    for (int32_t e = blk; e < a.E; e += nblk) {
+    const int nwarps = blockDim.x / kWarp;
+    const int warp = threadIdx.x / kWarp, lane = lane_id();
+    for (int32_t e = blk * nwarps + warp; e < E; e += nblk * nwarps) {
         int64_t lo = (int64_t)off[e] + cnt[e];
-        int64_t hi = off[e + 1] < a.rows_cap ? off[e + 1] : a.rows_cap;
-        for (int64_t r = lo + threadIdx.x; r < hi; r += kMetaThreads)
-            a.recv_src[r] = -1;
+        int64_t hi = off[e + 1] < rows_cap ? off[e + 1] : rows_cap;
+        for (int64_t r = lo + lane; r < hi; r += kWarp)
+            recv_src[r] = -1;
     }
-    for (int64_t r = (int64_t)off[a.E] + (int64_t)blk * kMetaThreads + threadIdx.x; r < a.rows_cap;
-         r += (int64_t)nblk * kMetaThreads)
-        a.recv_src[r] = -1;
+    for (int64_t r = (int64_t)off[E] + (int64_t)blk * blockDim.x + threadIdx.x; r < rows_cap;
+         r += (int64_t)nblk * blockDim.x)
+        recv_src[r] = -1;
 }
 
 // ---- one-CTA path -------------------------------------------------------------
@@ -211,7 +217,7 @@ __global__ void __launch_bounds__(kMetaThreads) meta_single_block(MetaArgs a)
         a.rank_offset[r] = off[(int64_t)r * (a.E / a.R)];
     __syncthreads();
     block_assign(a, 0, a.S, cursor, wcnt);
-    block_fill_unused(a, cnt, off, 0, 1);
+    block_fill_unused(a.rows_cap, a.E, a.recv_src, cnt, off, 0, 1);
 }
 
 // ---- tiled path ----------------------------------------------------------------
@@ -237,12 +243,21 @@ __global__ void __launch_bounds__(kMetaThreads) meta_tile_scan(MetaArgs a, int32
 {
     extern __shared__ int32_t sm[];
     int32_t *cnt = sm, *off = sm + a.E;
+    // One thread per expert walks the tiles; loads are issued 8 at a time so
+    // their latencies overlap.
     for (int32_t e = threadIdx.x; e < a.E; e += kMetaThreads) {
         int32_t run = 0;
-        for (int32_t t = 0; t < ntiles; ++t) {
-            int32_t c = tile_hist[(int64_t)t * a.E + e];
-            tile_hist[(int64_t)t * a.E + e] = run;
-            run += c;
+        for (int32_t t0 = 0; t0 < ntiles; t0 += 8) {
+            int32_t c[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                c[u] = t0 + u < ntiles ? tile_hist[(int64_t)(t0 + u) * a.E + e] : 0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (t0 + u < ntiles)
+                    tile_hist[(int64_t)(t0 + u) * a.E + e] = run;
+                run += c[u];
+            }
         }
         cnt[e] = run;
     }
@@ -274,7 +289,8 @@ __global__ void __launch_bounds__(kMetaThreads) meta_tile_assign(MetaArgs a,
     int64_t begin = (int64_t)blockIdx.x * kTileEntries;
     int64_t end = begin + kTileEntries < a.S ? begin + kTileEntries : a.S;
     block_assign(a, begin, end, cursor, wcnt);
-    block_fill_unused(a, a.expert_count, a.expert_offset, blockIdx.x, gridDim.x);
+    block_fill_unused(a.rows_cap, a.E, a.recv_src, a.expert_count, a.expert_offset,
+                                    blockIdx.x, gridDim.x);
 }
 
 inline size_t meta_single_smem(int32_t E) { return sizeof(int32_t) * ((size_t)3 * E + 1 + (size_t)kMetaWarps * E); }

@@ -10,6 +10,7 @@
 
 #include "combine.cuh"
 #include "common.cuh"
+#include "dispatch_fused.cuh"
 #include "meta.cuh"
 #include "scatter.cuh"
 
@@ -77,6 +78,37 @@ int64_t rows_capacity(const moe_config *c, int32_t T)
 }
 
 bool use_single_block(int64_t S) { return S <= kSingleBlockEntries; }
+
+// Vectors per thread of the fused small-batch dispatch, or 0 if it does not apply.
+int fused_vpt(const moe_config *c, int32_t T)
+{
+    const int64_t S = (int64_t)T * c->k;
+    const int32_t nvec = c->H / 8;
+    if (T <= 0 || S > kFusedMaxEntries || c->k > kFusedMaxK)
+        return 0;
+    for (int vpt = 1; vpt <= kFusedMaxVpt; vpt *= 2)
+        if (nvec <= kFusedMaxThreads * vpt)
+            return vpt;
+    return 0;
+}
+
+template <bool kFp8>
+cudaError_t launch_fused(int vpt, unsigned grid, unsigned block, size_t smem, cudaStream_t s,
+                         const FusedArgs &f)
+{
+    switch (vpt) {
+    case 1:
+        dispatch_fused<1, kFp8><<<grid, block, smem, s>>>(f);
+        break;
+    case 2:
+        dispatch_fused<2, kFp8><<<grid, block, smem, s>>>(f);
+        break;
+    default:
+        dispatch_fused<4, kFp8><<<grid, block, smem, s>>>(f);
+        break;
+    }
+    return cudaGetLastError();
+}
 
 size_t workspace_bytes(const moe_config *c, int32_t T)
 {
@@ -207,6 +239,39 @@ int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
     m.slot = slot;
     m.recv_src = out->recv_src;
     m.err = dev_err;
+
+    if (const int vpt = fused_vpt(cfg, T)) {
+        FusedArgs f;
+        f.x = static_cast<const uint16_t *>(x);
+        f.topk_idx = topk_idx;
+        f.T = T;
+        f.H = cfg->H;
+        f.k = cfg->k;
+        f.E = cfg->E;
+        f.R = cfg->R;
+        f.pad128 = m.pad128;
+        f.rows_cap = rows_cap;
+        f.recv_x = out->recv_x;
+        f.recv_scale = out->recv_scale;
+        f.expert_count = out->expert_count;
+        f.expert_offset = out->expert_offset;
+        f.rank_offset = out->rank_offset;
+        f.recv_src = out->recv_src;
+        f.slot = slot;
+        f.err = dev_err;
+        const int32_t nvec = cfg->H / 8;
+        const unsigned block = (unsigned)(((nvec + vpt - 1) / vpt + kWarp - 1) / kWarp * kWarp);
+        const cudaError_t e = fp8 ? launch_fused<true>(vpt, T, block, fused_smem(cfg->E), s, f)
+                                  : launch_fused<false>(vpt, T, block, fused_smem(cfg->E), s, f);
+        if ((st = launched(e)) != MOE_OK)
+            return st;
+        handle->cfg = *cfg;
+        handle->T = T;
+        handle->slot = slot;
+        handle->topk_w = topk_w;
+        handle->rows_cap = rows_cap;
+        return MOE_OK;
+    }
 
     if (use_single_block(S)) {
         meta_single_block<<<1, kMetaThreads, meta_single_smem(cfg->E), s>>>(m);
