@@ -6,7 +6,8 @@
 // Combinação"), shaped for decode batches where one launch and one DRAM round
 // trip cost more than the bytes.
 //
-// One CTA per token t.  The CTA first issues the loads of x[t] (they do not
+// One CTA per token t; its warps own the 512-column chunks of x[t] in the
+// scatter's layout.  The CTA first issues the loads of x[t] (they do not
 // depend on the routing), then reads all S = T*k expert ids (a few KB, served
 // from L2 after the first CTA) and builds in shared memory the histogram of all
 // entries and, in the same pass, the histogram of the entries that come before
@@ -29,7 +30,8 @@ namespace moe {
 constexpr int kFusedMaxEntries = 2048;
 constexpr int kFusedMaxK = 16;
 constexpr int kFusedMaxThreads = 512;
-constexpr int kFusedMaxVpt = 4; // 16-byte vectors per thread: rows up to 2048 vectors
+constexpr int kFusedMaxChunks = 4; // 512-column chunks per warp: rows up to 16 warps x 4 x 512
+constexpr int kFusedLoadRounds = 4; // expert ids loaded together per thread
 
 struct FusedArgs {
     const uint16_t *x;
@@ -45,28 +47,33 @@ struct FusedArgs {
 // Shared memory: hist[E], before[E], off[E+1].
 inline size_t fused_smem(int32_t E) { return sizeof(int32_t) * ((size_t)3 * E + 1); }
 
-template <int kVpt, bool kFp8>
+template <int kChunks, bool kFp8>
 __global__ void __launch_bounds__(kFusedMaxThreads) dispatch_fused(FusedArgs a)
 {
     extern __shared__ int32_t sm[];
     int32_t *hist = sm, *before = sm + a.E, *off = sm + 2 * a.E;
     __shared__ int32_t s_slot[kFusedMaxK];
+    __shared__ int32_t s_own[kFusedMaxK];
 
     const int32_t t = blockIdx.x;
     const int nt = blockDim.x;
+    const int nwarps = nt / kWarp;
+    const int warp = threadIdx.x / kWarp;
     const unsigned lane = lane_id();
-    const int32_t nvec = a.H / 8;
+    const int32_t chunks = (a.H + kChunkCols - 1) / kChunkCols;
 
-    // 1. The row's loads go out first.
-    uint4 val[kVpt];
+    // 1. The row's loads go out first: warp w owns chunks w, w + nwarps, ...
+    const uint16_t *xr = a.x + (int64_t)t * a.H;
+    uint4 v0[kChunks], v1[kChunks];
 #pragma unroll
-    for (int i = 0; i < kVpt; ++i) {
-        const int32_t v = threadIdx.x + i * nt;
-        val[i] = v < nvec ? ld_stream_v4(a.x + (int64_t)t * a.H + (int64_t)v * 8)
-                          : make_uint4(0u, 0u, 0u, 0u);
+    for (int i = 0; i < kChunks; ++i) {
+        const int32_t c = warp + i * nwarps;
+        if (c < chunks)
+            load_chunk<kFp8>(xr, a.H, c, v0[i], v1[i]);
     }
 
-    // 2. Histograms of all entries and of the entries before token t.
+    // 2. Histograms of all entries and of the entries before token t; the
+    //    token's own ids are kept in shared memory.
     for (int32_t e = threadIdx.x; e < a.E; e += nt) {
         hist[e] = 0;
         before[e] = 0;
@@ -74,24 +81,32 @@ __global__ void __launch_bounds__(kFusedMaxThreads) dispatch_fused(FusedArgs a)
     __syncthreads();
     const int64_t S = (int64_t)a.T * a.k;
     const int64_t mine = (int64_t)t * a.k;
-    for (int64_t base = 0; base < S; base += nt) {
-        const int64_t i = base + threadIdx.x;
-        int32_t e = -1;
-        if (i < S) {
-            e = __ldg(a.topk_idx + i);
-            if (e < 0 || e >= a.E) {
+    for (int64_t base = 0; base < S; base += (int64_t)nt * kFusedLoadRounds) {
+        int32_t ev[kFusedLoadRounds];
+#pragma unroll
+        for (int r = 0; r < kFusedLoadRounds; ++r) {
+            const int64_t i = base + (int64_t)r * nt + threadIdx.x;
+            ev[r] = i < S ? __ldg(a.topk_idx + i) : -1;
+        }
+#pragma unroll
+        for (int r = 0; r < kFusedLoadRounds; ++r) {
+            const int64_t i = base + (int64_t)r * nt + threadIdx.x;
+            int32_t e = ev[r];
+            if (i >= mine && i < mine + a.k)
+                s_own[i - mine] = e;
+            if (i < S && (e < 0 || e >= a.E)) {
                 if (t == 0)
                     raise_error(a.err, MOE_DEV_BAD_INDEX);
                 e = -1;
             }
-        }
-        const unsigned peers = __match_any_sync(kFullMask, e);
-        const unsigned below = __ballot_sync(kFullMask, i < mine);
-        if (e >= 0 && lane == (unsigned)(__ffs(peers) - 1)) {
-            atomicAdd(&hist[e], __popc(peers));
-            const int nb = __popc(peers & below);
-            if (nb)
-                atomicAdd(&before[e], nb);
+            const unsigned peers = __match_any_sync(kFullMask, e);
+            const unsigned below = __ballot_sync(kFullMask, i < mine);
+            if (e >= 0 && lane == (unsigned)(__ffs(peers) - 1)) {
+                atomicAdd(&hist[e], __popc(peers));
+                const int nb = __popc(peers & below);
+                if (nb)
+                    atomicAdd(&before[e], nb);
+            }
         }
     }
     __syncthreads();
@@ -102,12 +117,12 @@ __global__ void __launch_bounds__(kFusedMaxThreads) dispatch_fused(FusedArgs a)
     // 4. This token's slots.
     if (threadIdx.x < a.k) {
         const int j = threadIdx.x;
-        const int32_t e = __ldg(a.topk_idx + mine + j);
+        const int32_t e = s_own[j];
         int32_t s = -1;
         if (e >= 0 && e < a.E) {
             int32_t dup = 0;
             for (int jj = 0; jj < j; ++jj)
-                dup += __ldg(a.topk_idx + mine + jj) == e;
+                dup += s_own[jj] == e;
             const int64_t row = (int64_t)off[e] + before[e] + dup;
             if (row < a.rows_cap) {
                 s = (int32_t)row;
@@ -133,38 +148,11 @@ __global__ void __launch_bounds__(kFusedMaxThreads) dispatch_fused(FusedArgs a)
     __syncthreads();
 
     // 5. Payload to the k slots.
-    if constexpr (kFp8) {
-        uint8_t *rx = static_cast<uint8_t *>(a.recv_x);
-        const int32_t nb = a.H / 128;
 #pragma unroll
-        for (int i = 0; i < kVpt; ++i) {
-            const int32_t v = threadIdx.x + i * nt;
-            float scale;
-            const uint2 codes = quantise_vec_e4m3(val[i], scale);
-            if (v >= nvec)
-                continue;
-            for (int32_t j = 0; j < a.k; ++j) {
-                const int32_t s = s_slot[j];
-                if (s < 0)
-                    continue;
-                st_v2(rx + (int64_t)s * a.H + (int64_t)v * 8, codes);
-                if ((lane & 15) == 0)
-                    a.recv_scale[(int64_t)s * nb + v / 16] = scale;
-            }
-        }
-    } else {
-        uint16_t *rx = static_cast<uint16_t *>(a.recv_x);
-        for (int32_t j = 0; j < a.k; ++j) {
-            const int32_t s = s_slot[j];
-            if (s < 0)
-                continue;
-#pragma unroll
-            for (int i = 0; i < kVpt; ++i) {
-                const int32_t v = threadIdx.x + i * nt;
-                if (v < nvec)
-                    st_v4(rx + (int64_t)s * a.H + (int64_t)v * 8, val[i]);
-            }
-        }
+    for (int i = 0; i < kChunks; ++i) {
+        const int32_t c = warp + i * nwarps;
+        if (c < chunks)
+            store_chunk<kFp8>(a.recv_x, a.recv_scale, a.H, c, a.k, s_slot, v0[i], v1[i]);
     }
 }
 

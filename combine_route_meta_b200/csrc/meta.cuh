@@ -20,13 +20,17 @@
 // + rank inside its own warp's group.
 // That is exactly the stable order, with no sort and no global atomics.
 //
-// Two launch shapes:
-//  - small batches (S <= kSingleBlockEntries): one CTA does counts, scan and
-//    slots in shared memory (one launch, no scratch);
-//  - large batches: tiles of kTileEntries entries.  (1) each CTA counts its
-//    tile into scratch tile_hist[tile][E]; (2) one CTA turns those into
-//    per-tile prefixes, the counts and the offsets; (3) each CTA re-reads its
-//    tile and assigns slots from offset[e] + tile prefix.
+// Launch shapes (small decode batches take the fused kernel in
+// dispatch_fused.cuh instead):
+//  - S <= kSingleBlockEntries: one CTA does counts, scan and slots in shared
+//    memory (one launch, no scratch);
+//  - larger batches: tiles of kTileEntries entries.  (1) each CTA counts its
+//    tile into scratch tile_hist[tile][E]; (2) CTAs of 32 experts turn each
+//    expert's column into an exclusive prefix over tiles and write the counts;
+//    (3) each CTA takes the scan of the counts for the offsets and assigns its
+//    tile's slots from offset[e] + tile prefix.
+// Every CTA loads the expert ids of all its rounds before the first round, so
+// it pays one memory latency, not one per round.
 #pragma once
 
 #include "common.cuh"
@@ -35,7 +39,7 @@ namespace moe {
 
 constexpr int kMetaThreads = 512;
 constexpr int kMetaWarps = kMetaThreads / kWarp;
-constexpr int kTileEntries = 2048;
+constexpr int kTileEntries = 1024;
 constexpr int kSingleBlockEntries = 4096;
 
 struct MetaArgs {
@@ -65,17 +69,35 @@ __device__ __forceinline__ int32_t entry_expert(const MetaArgs &a, int64_t i, bo
     return e;
 }
 
-// Adds the entries [begin, end) into hist[E] (shared memory).
+// Expert ids of entries begin + r*kMetaThreads + threadIdx.x for r < kRounds
+// (-1 where there is no entry), loaded together.
+template <int kRounds>
+__device__ __forceinline__ void load_entries(const MetaArgs &a, int64_t begin, int64_t end,
+                                             bool flag_bad, int32_t (&e)[kRounds])
+{
+#pragma unroll
+    for (int r = 0; r < kRounds; ++r) {
+        const int64_t i = begin + (int64_t)r * kMetaThreads + threadIdx.x;
+        e[r] = i < end ? entry_expert(a, i, flag_bad) : -1;
+    }
+}
+
+// Adds the entries [begin, end) into hist[E] (shared memory);
+// end - begin <= kRounds * kMetaThreads.
+template <int kRounds>
 __device__ __forceinline__ void block_count(const MetaArgs &a, int64_t begin, int64_t end,
                                             int32_t *hist)
 {
+    int32_t e[kRounds];
+    load_entries<kRounds>(a, begin, end, true, e);
     const unsigned lane = lane_id();
-    for (int64_t base = begin; base < end; base += kMetaThreads) {
-        int64_t i = base + threadIdx.x;
-        int32_t e = i < end ? entry_expert(a, i, true) : -1;
-        unsigned peers = __match_any_sync(kFullMask, e);
-        if (e >= 0 && lane == (unsigned)(__ffs(peers) - 1))
-            atomicAdd(&hist[e], __popc(peers));
+#pragma unroll
+    for (int r = 0; r < kRounds; ++r) {
+        if (begin + (int64_t)r * kMetaThreads >= end)
+            break;
+        const unsigned peers = __match_any_sync(kFullMask, e[r]);
+        if (e[r] >= 0 && lane == (unsigned)(__ffs(peers) - 1))
+            atomicAdd(&hist[e[r]], __popc(peers));
     }
 }
 
@@ -125,21 +147,29 @@ __device__ void block_offsets(const int32_t *cnt, int32_t *off, int32_t E, int32
     __syncthreads();
 }
 
-// Assigns slots to entries [begin, end) in order.  cursor[e] (shared) holds the
-// first free row of expert e for this range and is advanced; wcnt is
-// [kMetaWarps][E] shared scratch that must be zero on entry and is zero on exit.
+// Assigns slots to entries [begin, end) in order; end - begin <= kRounds *
+// kMetaThreads.  cursor[e] (shared) holds the first free row of expert e for
+// this range and is advanced; wcnt is [kMetaWarps][E] shared scratch that must
+// be zero on entry and is zero on exit.
+template <int kRounds>
 __device__ __forceinline__ void block_assign(const MetaArgs &a, int64_t begin, int64_t end,
                                              int32_t *cursor, int32_t *wcnt)
 {
+    int32_t ev[kRounds];
+    load_entries<kRounds>(a, begin, end, false, ev);
     const unsigned lane = lane_id(), warp = threadIdx.x / kWarp;
-    for (int64_t base = begin; base < end; base += kMetaThreads) {
-        int64_t i = base + threadIdx.x;
-        int32_t e = i < end ? entry_expert(a, i, false) : -1;
-        unsigned peers = __match_any_sync(kFullMask, e);
-        unsigned leader = __ffs(peers) - 1;
-        int32_t rank = __popc(peers & lanemask_lt());
-        int32_t group = __popc(peers);
-        bool lead = e >= 0 && lane == leader;
+#pragma unroll
+    for (int r = 0; r < kRounds; ++r) {
+        const int64_t base = begin + (int64_t)r * kMetaThreads;
+        if (base >= end)
+            break;
+        const int64_t i = base + threadIdx.x;
+        const int32_t e = ev[r];
+        const unsigned peers = __match_any_sync(kFullMask, e);
+        const unsigned leader = __ffs(peers) - 1;
+        const int32_t rank = __popc(peers & lanemask_lt());
+        const int32_t group = __popc(peers);
+        const bool lead = e >= 0 && lane == leader;
         if (lead)
             wcnt[warp * a.E + e] = group;
         __syncthreads();
@@ -158,7 +188,7 @@ __device__ __forceinline__ void block_assign(const MetaArgs &a, int64_t begin, i
         if (i < end) {
             int32_t s = -1;
             if (e >= 0) {
-                int64_t row = (int64_t)first + rank;
+                const int64_t row = (int64_t)first + rank;
                 if (row < a.rows_cap) {
                     s = (int32_t)row;
                     a.recv_src[row] = (int32_t)i;
@@ -192,7 +222,23 @@ __device__ __forceinline__ void block_fill_unused(int64_t rows_cap, int32_t E, i
         recv_src[r] = -1;
 }
 
+// Writes expert_count, expert_offset and rank_offset from shared cnt/off.
+__device__ __forceinline__ void write_offsets(const MetaArgs &a, const int32_t *cnt,
+                                              const int32_t *off)
+{
+    for (int32_t e = threadIdx.x; e < a.E; e += blockDim.x) {
+        a.expert_count[e] = cnt[e];
+        a.expert_offset[e] = off[e];
+    }
+    if (threadIdx.x == 0)
+        a.expert_offset[a.E] = off[a.E];
+    for (int32_t r = threadIdx.x; r <= a.R; r += blockDim.x)
+        a.rank_offset[r] = off[(int64_t)r * (a.E / a.R)];
+}
+
 // ---- one-CTA path -------------------------------------------------------------
+constexpr int kSingleRounds = kSingleBlockEntries / kMetaThreads;
+
 // Shared memory: cnt[E], off[E+1], cursor[E], wcnt[kMetaWarps*E].
 __global__ void __launch_bounds__(kMetaThreads) meta_single_block(MetaArgs a)
 {
@@ -203,24 +249,20 @@ __global__ void __launch_bounds__(kMetaThreads) meta_single_block(MetaArgs a)
     for (int32_t i = threadIdx.x; i < kMetaWarps * a.E; i += kMetaThreads)
         wcnt[i] = 0;
     __syncthreads();
-    block_count(a, 0, a.S, cnt);
+    block_count<kSingleRounds>(a, 0, a.S, cnt);
     __syncthreads();
     block_offsets(cnt, off, a.E, a.pad128);
-    for (int32_t e = threadIdx.x; e < a.E; e += kMetaThreads) {
+    write_offsets(a, cnt, off);
+    for (int32_t e = threadIdx.x; e < a.E; e += kMetaThreads)
         cursor[e] = off[e];
-        a.expert_count[e] = cnt[e];
-        a.expert_offset[e] = off[e];
-    }
-    if (threadIdx.x == 0)
-        a.expert_offset[a.E] = off[a.E];
-    for (int32_t r = threadIdx.x; r <= a.R; r += kMetaThreads)
-        a.rank_offset[r] = off[(int64_t)r * (a.E / a.R)];
     __syncthreads();
-    block_assign(a, 0, a.S, cursor, wcnt);
+    block_assign<kSingleRounds>(a, 0, a.S, cursor, wcnt);
     block_fill_unused(a.rows_cap, a.E, a.recv_src, cnt, off, 0, 1);
 }
 
 // ---- tiled path ----------------------------------------------------------------
+constexpr int kTileRounds = kTileEntries / kMetaThreads;
+
 // (1) tile_hist[tile][e] = entries of tile `tile` routed to e.
 __global__ void __launch_bounds__(kMetaThreads) meta_tile_count(MetaArgs a, int32_t *tile_hist)
 {
@@ -228,75 +270,97 @@ __global__ void __launch_bounds__(kMetaThreads) meta_tile_count(MetaArgs a, int3
     for (int32_t e = threadIdx.x; e < a.E; e += kMetaThreads)
         hist[e] = 0;
     __syncthreads();
-    int64_t begin = (int64_t)blockIdx.x * kTileEntries;
-    int64_t end = begin + kTileEntries < a.S ? begin + kTileEntries : a.S;
-    block_count(a, begin, end, hist);
+    const int64_t begin = (int64_t)blockIdx.x * kTileEntries;
+    const int64_t end = begin + kTileEntries < a.S ? begin + kTileEntries : a.S;
+    block_count<kTileRounds>(a, begin, end, hist);
     __syncthreads();
     for (int32_t e = threadIdx.x; e < a.E; e += kMetaThreads)
         tile_hist[(int64_t)blockIdx.x * a.E + e] = hist[e];
 }
 
-// (2) One CTA: tile_hist becomes the exclusive prefix over tiles (per expert),
-// and the counts, offsets and rank offsets are written.
-__global__ void __launch_bounds__(kMetaThreads) meta_tile_scan(MetaArgs a, int32_t *tile_hist,
+// (2) Per-expert exclusive prefix over tiles, in place, and the counts.
+// A CTA owns 32 experts (one per lane); its 8 warps split the tiles, add their
+// share, combine the shares through shared memory, then rewrite their tiles
+// with running prefixes.  Loads are issued 8 tiles at a time.
+constexpr int kScanThreads = 256;
+constexpr int kScanWarps = kScanThreads / kWarp;
+
+__global__ void __launch_bounds__(kScanThreads) meta_tile_scan(MetaArgs a, int32_t *tile_hist,
                                                                int32_t ntiles)
 {
-    extern __shared__ int32_t sm[];
-    int32_t *cnt = sm, *off = sm + a.E;
-    // One thread per expert walks the tiles; loads are issued 8 at a time so
-    // their latencies overlap.
-    for (int32_t e = threadIdx.x; e < a.E; e += kMetaThreads) {
-        int32_t run = 0;
-        for (int32_t t0 = 0; t0 < ntiles; t0 += 8) {
-            int32_t c[8];
+    __shared__ int32_t part[kScanWarps][kWarp];
+    const int warp = threadIdx.x / kWarp, lane = lane_id();
+    const int32_t e = blockIdx.x * kWarp + lane;
+    const bool valid = e < a.E;
+    const int32_t per = (ntiles + kScanWarps - 1) / kScanWarps;
+    const int32_t t_lo = warp * per;
+    const int32_t t_hi = t_lo + per < ntiles ? t_lo + per : ntiles;
+    int32_t sum = 0;
+    for (int32_t t0 = t_lo; t0 < t_hi; t0 += 8) {
+        int32_t c[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                c[u] = t0 + u < ntiles ? tile_hist[(int64_t)(t0 + u) * a.E + e] : 0;
+        for (int u = 0; u < 8; ++u)
+            c[u] = (valid && t0 + u < t_hi) ? tile_hist[(int64_t)(t0 + u) * a.E + e] : 0;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                if (t0 + u < ntiles)
-                    tile_hist[(int64_t)(t0 + u) * a.E + e] = run;
-                run += c[u];
-            }
-        }
-        cnt[e] = run;
+        for (int u = 0; u < 8; ++u)
+            sum += c[u];
     }
+    part[warp][lane] = sum;
     __syncthreads();
-    block_offsets(cnt, off, a.E, a.pad128);
-    for (int32_t e = threadIdx.x; e < a.E; e += kMetaThreads) {
-        a.expert_count[e] = cnt[e];
-        a.expert_offset[e] = off[e];
+    int32_t run = 0, total = 0;
+    for (int w = 0; w < kScanWarps; ++w) {
+        if (w < warp)
+            run += part[w][lane];
+        total += part[w][lane];
     }
-    if (threadIdx.x == 0)
-        a.expert_offset[a.E] = off[a.E];
-    for (int32_t r = threadIdx.x; r <= a.R; r += kMetaThreads)
-        a.rank_offset[r] = off[(int64_t)r * (a.E / a.R)];
+    for (int32_t t0 = t_lo; t0 < t_hi; t0 += 8) {
+        int32_t c[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            c[u] = (valid && t0 + u < t_hi) ? tile_hist[(int64_t)(t0 + u) * a.E + e] : 0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            if (valid && t0 + u < t_hi)
+                tile_hist[(int64_t)(t0 + u) * a.E + e] = run;
+            run += c[u];
+        }
+    }
+    if (valid && warp == 0)
+        a.expert_count[e] = total;
 }
 
-// (3) Slots of one tile, from offset[e] + the tile's prefix; also clears the
-// unused rows' recv_src (split over all CTAs).
-// Shared memory: cursor[E], wcnt[kMetaWarps*E].
+// (3) Slots of one tile.  Every CTA scans the counts for the offsets (E values,
+// cheaper than another launch), starts each expert's cursor at offset[e] + the
+// tile's prefix, and assigns its entries; CTA 0 writes the offsets, and all
+// CTAs share clearing the unused rows' recv_src.
+// Shared memory: cnt[E], off[E+1], cursor[E], wcnt[kMetaWarps*E].
 __global__ void __launch_bounds__(kMetaThreads) meta_tile_assign(MetaArgs a,
                                                                  const int32_t *tile_prefix)
 {
     extern __shared__ int32_t sm[];
-    int32_t *cursor = sm, *wcnt = sm + a.E;
-    for (int32_t e = threadIdx.x; e < a.E; e += kMetaThreads)
-        cursor[e] = a.expert_offset[e] + tile_prefix[(int64_t)blockIdx.x * a.E + e];
+    int32_t *cnt = sm, *off = sm + a.E, *cursor = off + a.E + 1, *wcnt = cursor + a.E;
+    for (int32_t e = threadIdx.x; e < a.E; e += kMetaThreads) {
+        cnt[e] = a.expert_count[e];
+        cursor[e] = tile_prefix[(int64_t)blockIdx.x * a.E + e];
+    }
     for (int32_t i = threadIdx.x; i < kMetaWarps * a.E; i += kMetaThreads)
         wcnt[i] = 0;
     __syncthreads();
-    int64_t begin = (int64_t)blockIdx.x * kTileEntries;
-    int64_t end = begin + kTileEntries < a.S ? begin + kTileEntries : a.S;
-    block_assign(a, begin, end, cursor, wcnt);
-    block_fill_unused(a.rows_cap, a.E, a.recv_src, a.expert_count, a.expert_offset,
-                                    blockIdx.x, gridDim.x);
+    block_offsets(cnt, off, a.E, a.pad128);
+    if (blockIdx.x == 0)
+        write_offsets(a, cnt, off);
+    for (int32_t e = threadIdx.x; e < a.E; e += kMetaThreads)
+        cursor[e] += off[e];
+    __syncthreads();
+    const int64_t begin = (int64_t)blockIdx.x * kTileEntries;
+    const int64_t end = begin + kTileEntries < a.S ? begin + kTileEntries : a.S;
+    block_assign<kTileRounds>(a, begin, end, cursor, wcnt);
+    block_fill_unused(a.rows_cap, a.E, a.recv_src, cnt, off, blockIdx.x, gridDim.x);
 }
 
 inline size_t meta_single_smem(int32_t E) { return sizeof(int32_t) * ((size_t)3 * E + 1 + (size_t)kMetaWarps * E); }
 inline size_t meta_count_smem(int32_t E) { return sizeof(int32_t) * (size_t)E; }
-inline size_t meta_scan_smem(int32_t E) { return sizeof(int32_t) * ((size_t)2 * E + 1); }
-inline size_t meta_assign_smem(int32_t E) { return sizeof(int32_t) * ((size_t)E + (size_t)kMetaWarps * E); }
+inline size_t meta_assign_smem(int32_t E) { return meta_single_smem(E); }
 
 inline int64_t meta_tiles(int64_t S) { return (S + kTileEntries - 1) / kTileEntries; }
 

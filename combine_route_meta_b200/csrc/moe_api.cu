@@ -79,24 +79,28 @@ int64_t rows_capacity(const moe_config *c, int32_t T)
 
 bool use_single_block(int64_t S) { return S <= kSingleBlockEntries; }
 
-// Vectors per thread of the fused small-batch dispatch, or 0 if it does not apply.
-int fused_vpt(const moe_config *c, int32_t T)
+// Chunks per warp of the fused small-batch dispatch (1, 2 or 4), or 0 if the
+// fused kernel does not apply.  *threads receives its block size.
+int fused_chunks(const moe_config *c, int32_t T, unsigned *threads)
 {
     const int64_t S = (int64_t)T * c->k;
-    const int32_t nvec = c->H / 8;
+    const int32_t chunks = (c->H + kChunkCols - 1) / kChunkCols;
     if (T <= 0 || S > kFusedMaxEntries || c->k > kFusedMaxK)
         return 0;
-    for (int vpt = 1; vpt <= kFusedMaxVpt; vpt *= 2)
-        if (nvec <= kFusedMaxThreads * vpt)
-            return vpt;
+    const int max_warps = kFusedMaxThreads / kWarp;
+    for (int per = 1; per <= kFusedMaxChunks; per *= 2)
+        if (chunks <= max_warps * per) {
+            *threads = (unsigned)((chunks + per - 1) / per) * kWarp;
+            return per;
+        }
     return 0;
 }
 
 template <bool kFp8>
-cudaError_t launch_fused(int vpt, unsigned grid, unsigned block, size_t smem, cudaStream_t s,
+cudaError_t launch_fused(int per, unsigned grid, unsigned block, size_t smem, cudaStream_t s,
                          const FusedArgs &f)
 {
-    switch (vpt) {
+    switch (per) {
     case 1:
         dispatch_fused<1, kFp8><<<grid, block, smem, s>>>(f);
         break;
@@ -240,7 +244,8 @@ int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
     m.recv_src = out->recv_src;
     m.err = dev_err;
 
-    if (const int vpt = fused_vpt(cfg, T)) {
+    unsigned fused_block = 0;
+    if (const int per = fused_chunks(cfg, T, &fused_block)) {
         FusedArgs f;
         f.x = static_cast<const uint16_t *>(x);
         f.topk_idx = topk_idx;
@@ -259,10 +264,9 @@ int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
         f.recv_src = out->recv_src;
         f.slot = slot;
         f.err = dev_err;
-        const int32_t nvec = cfg->H / 8;
-        const unsigned block = (unsigned)(((nvec + vpt - 1) / vpt + kWarp - 1) / kWarp * kWarp);
-        const cudaError_t e = fp8 ? launch_fused<true>(vpt, T, block, fused_smem(cfg->E), s, f)
-                                  : launch_fused<false>(vpt, T, block, fused_smem(cfg->E), s, f);
+        const cudaError_t e =
+            fp8 ? launch_fused<true>(per, T, fused_block, fused_smem(cfg->E), s, f)
+                : launch_fused<false>(per, T, fused_block, fused_smem(cfg->E), s, f);
         if ((st = launched(e)) != MOE_OK)
             return st;
         handle->cfg = *cfg;
@@ -281,7 +285,8 @@ int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
         const int64_t ntiles = meta_tiles(S);
         int32_t *tile_hist = static_cast<int32_t *>(workspace);
         meta_tile_count<<<(unsigned)ntiles, kMetaThreads, meta_count_smem(cfg->E), s>>>(m, tile_hist);
-        meta_tile_scan<<<1, kMetaThreads, meta_scan_smem(cfg->E), s>>>(m, tile_hist, (int32_t)ntiles);
+        meta_tile_scan<<<(unsigned)((cfg->E + kWarp - 1) / kWarp), kScanThreads, 0, s>>>(
+            m, tile_hist, (int32_t)ntiles);
         meta_tile_assign<<<(unsigned)ntiles, kMetaThreads, meta_assign_smem(cfg->E), s>>>(m, tile_hist);
         if ((st = launched(cudaGetLastError())) != MOE_OK)
             return st;
@@ -294,10 +299,12 @@ int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
         a.T = T;
         a.H = cfg->H;
         a.k = cfg->k;
-        a.parts = (cfg->H / 8 + kScatterThreads - 1) / kScatterThreads;
         a.recv_x = out->recv_x;
         a.recv_scale = out->recv_scale;
-        const unsigned grid = grid_for((int64_t)T * a.parts, dev->sms, 16);
+        const int64_t warp_units = (int64_t)T * ((cfg->H + kChunkCols - 1) / kChunkCols);
+        const int warps_per_cta = kScatterThreads / kWarp;
+        const unsigned grid =
+            grid_for((warp_units + warps_per_cta - 1) / warps_per_cta, dev->sms, 2048 / kScatterThreads);
         if (fp8)
             scatter_rows<true><<<grid, kScatterThreads, 0, s>>>(a);
         else

@@ -160,13 +160,16 @@ def test_workload_parity_sampled_largest():
 
 CASES = [
     # T, H, E, R, k, fp8, pad128, distinct
-    # fused one-launch dispatch (S <= 2048, k <= 16): 1, 2 and 4 vectors per thread
+    # fused one-launch dispatch (S <= 2048, k <= 16): 1, 2 and 4 chunks per warp
     (1, 8, 1, 1, 1, False, False, True),
     (64, 7168, 32, 4, 8, False, True, True),
     (3, 16384, 16, 4, 4, True, False, True),
+    (2, 24576, 16, 4, 4, True, True, True),
     (256, 7168, 256, 32, 8, True, True, True),   # S = 2048: the largest fused batch
     # one-CTA metadata + scatter: k > 16, or 2048 < S <= 4096
     (10, 128, 8, 2, 20, False, False, False),
+    (600, 1032, 16, 4, 5, False, True, False),   # ragged last 512-column chunk (8 columns)
+    (300, 1152, 8, 8, 8, True, True, True),      # 9 scales per row: no 16-byte scale stores
     (1, 128, 4, 2, 4, True, False, True),
     (5, 136, 6, 3, 3, False, False, True),       # H/8 = 17 vectors: one ragged part
     (33, 1032, 16, 4, 5, False, True, False),    # 129 vectors: two parts, duplicates
