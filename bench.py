@@ -207,82 +207,114 @@ def time_oracle(w, budget_s=10.0, max_reps=50):
 
 # ---- GPU arm ----------------------------------------------------------------------------
 
+def count_graph_kernels(g):
+    """Kernel nodes in a captured torch CUDA graph (the launches of one replay)."""
+    from cuda.bindings import runtime as rt
+    graph = rt.cudaGraph_t(init_value=g.raw_cuda_graph())
+    err, _, n = rt.cudaGraphGetNodes(graph, 0)
+    if err != rt.cudaError_t.cudaSuccess:
+        raise RuntimeError(f"cudaGraphGetNodes: {err}")
+    err, nodes, n = rt.cudaGraphGetNodes(graph, n)
+    kernels = 0
+    for node in nodes[:n]:
+        err, kind = rt.cudaGraphNodeGetType(node)
+        if kind == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+            kernels += 1
+    return kernels
+
+
 def run_gpu(args, rank, world):
+    import dataclasses
+    import math
+
     import torch
     import combine_route_meta_b200 as moe
     from workloads import WORKLOADS, make_expert_out, make_inputs
 
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
-    w = WORKLOADS[args.workload]
-    import dataclasses
-    w = dataclasses.replace(w, seed=w.seed + rank)
+    w = dataclasses.replace(WORKLOADS[args.workload], seed=WORKLOADS[args.workload].seed + rank)
+    if w.identity_experts and w.fp8:
+        raise SystemExit("identity experts need a bf16 dispatch")
     _, x, idx, wts = make_inputs(w)
     cfg = moe.make_config(w.H, w.k, w.E, w.R, w.fp8, w.pad128)
-    buf = moe.Buffers(cfg, w.T, dev)
-    eo_host = make_expert_out(w, buf.rows_cap)
+    rows_cap = moe.rows_capacity(cfg, w.T)
+    eo_host = None if w.identity_experts else make_expert_out(w, rows_cap)
 
     def bf16_dev(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
 
-    xd, idd, wd = bf16_dev(x), torch.from_numpy(idx).to(dev), torch.from_numpy(wts).to(dev)
-    eo = buf.recv_x if w.identity_experts else bf16_dev(eo_host)
-    if w.identity_experts and w.fp8:
-        raise SystemExit("identity experts need a bf16 dispatch")
-    y = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev)
-
-    # L2 flush between steps: write a 2x-L2 buffer, then read another 2x-L2 buffer,
-    # so the step starts with no payload lines cached and no dirty lines to evict.
+    # Inputs larger than L2 between uses of the same bytes: rotate through enough
+    # independent sets (inputs and outputs) that one step's data is evicted
+    # before it comes round again.
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush_w = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
-    flush_r = torch.zeros(2 * l2 // 4, dtype=torch.int32, device=dev)
-    flush_sink = torch.empty((), dtype=torch.int64, device=dev)
+    recv_bytes = rows_cap * w.H * (1 if w.fp8 else 2) + (rows_cap * (w.H // 128) * 4 if w.fp8 else 0)
+    set_bytes = (x.nbytes + idx.nbytes + wts.nbytes + (0 if eo_host is None else eo_host.nbytes)
+                 + recv_bytes + rows_cap * 4 + idx.nbytes + w.T * w.H * 2)
+    nsets = 1 if set_bytes >= 2 * l2 else math.ceil(2 * l2 / set_bytes) + 1
+
+    class Set:
+        pass
+
+    sets = []
+    for _ in range(nsets):
+        st = Set()
+        st.buf = moe.Buffers(cfg, w.T, dev)
+        st.x, st.idx, st.w = bf16_dev(x), torch.from_numpy(idx).to(dev), torch.from_numpy(wts).to(dev)
+        st.eo = st.buf.recv_x if eo_host is None else bf16_dev(eo_host)
+        st.y = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev)
+        sets.append(st)
     stream = torch.cuda.Stream(device=dev)
 
-    def do_dispatch():
-        moe.dispatch_into(buf, xd, idd, wd, stream=stream)
+    def do_dispatch(st):
+        moe.dispatch_into(st.buf, st.x, st.idx, st.w, stream=stream)
 
-    def do_combine():
-        moe.combine_into(buf.handle_c, eo, y, buf.err, stream=stream)
+    def do_combine(st):
+        moe.combine_into(st.buf.handle_c, st.eo, st.y, st.buf.err, stream=stream)
 
-    # warm-up (also loads the kernels) and graph capture on a side stream
     with torch.cuda.stream(stream):
-        for _ in range(2):
-            do_dispatch()
-            do_combine()
+        for st in sets:
+            do_dispatch(st)
+            do_combine(st)
     stream.synchronize()
-    g_disp, g_comb = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_disp, stream=stream):
-        do_dispatch()
-    with torch.cuda.graph(g_comb, stream=stream):
-        do_combine()
     if moe.check(stream) != 0:
         raise RuntimeError("device error during warm-up")
 
-    launches_per_step = (1 if moe.workspace_bytes(cfg, w.T) == 0 else 3) + 1 + 1
+    # One CUDA graph per set and phase (the step graph holds dispatch + combine).
+    def capture(fn):
+        g = torch.cuda.CUDAGraph(keep_graph=True)
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        return g
 
-    def step(evs):
+    g_step = [capture(lambda st=st: (do_dispatch(st), do_combine(st))) for st in sets]
+    g_disp = [capture(lambda st=st: do_dispatch(st)) for st in sets]
+    g_comb = [capture(lambda st=st: do_combine(st)) for st in sets]
+    launches_per_step = count_graph_kernels(g_step[0])
+    for g in g_step + g_disp + g_comb:
+        g.instantiate()
+
+    def run(graphs, n):
+        """Replays n graphs back to back (rotating sets); device milliseconds."""
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
-            flush_w.zero_()
-            torch.sum(flush_r, dim=0, dtype=torch.int64, out=flush_sink)
-            torch.cuda._sleep(20_000)  # lets the host queue the step before the GPU reaches it
-            evs[0].record(stream)
-            g_disp.replay()
-            evs[1].record(stream)
-            g_comb.replay()
-            evs[2].record(stream)
+            # a sleeping kernel in front lets the host queue the replays ahead of the GPU
+            torch.cuda._sleep(min(n, 256) * 20_000)
+            e0.record(stream)
+            for i in range(n):
+                graphs[i % nsets].replay()
+            e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1)
 
     # Warm-up: at least W steps, and on until the clock sampler reports (the GPU
     # is then under load when the timed region starts).
     sampler = ClockSampler(dev.index)
     sampler.start()
     t_warm = time.monotonic()
-    n = 0
-    while n < args.warmup or (sampler.count() < 2 and time.monotonic() - t_warm < 5.0):
-        step([torch.cuda.Event(enable_timing=True) for _ in range(3)])
-        n += 1
-        if n % 20 == 0:
-            torch.cuda.synchronize()
+    run(g_step, max(args.warmup, nsets))
+    while sampler.count() < 3 and time.monotonic() - t_warm < 5.0:
+        run(g_step, 200)
     torch.cuda.synchronize()
 
     dist = None
@@ -291,36 +323,33 @@ def run_gpu(args, rank, world):
         dist.barrier()
     torch.cuda.synchronize()
     sampler.mark_start()
-    all_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    for evs in all_evs:
-        step(evs)
+    total_ms = run(g_step, args.steps)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     sampler.mark_end()
     clocks = sampler.stop()
-
-    disp_ms = [a.elapsed_time(b) for a, b, _ in all_evs]
-    comb_ms = [b.elapsed_time(c) for _, b, c in all_evs]
-    step_ms = [a.elapsed_time(c) for a, _, c in all_evs]
     bits = moe.check(stream)
     if bits:
         raise RuntimeError(f"device error bits {bits} during timing")
-
-    total_ms = sum(step_ms)
     if dist is not None:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
 
-    # end-to-end through the public API with host buffers: H2D of the step's inputs,
-    # dispatch, combine, D2H of y, every step
+    # Phase split, same protocol: K dispatches alone, then K combines alone.
+    disp_ms = run(g_disp, args.steps)
+    comb_ms = run(g_comb, args.steps)
+
+    # End to end through the public API with host buffers: H2D of the step's
+    # inputs, dispatch, combine, D2H of y, every step.
+    st = sets[0]
     pin = dict(pin_memory=True)
     x_h = torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).pin_memory()
     idx_h = torch.from_numpy(idx).pin_memory()
     w_h = torch.from_numpy(wts).pin_memory()
-    eo_h = (None if w.identity_experts else
+    eo_h = (None if eo_host is None else
             torch.from_numpy(np.ascontiguousarray(eo_host).view(np.int16)).view(torch.bfloat16).pin_memory())
     y_h = torch.empty((w.T, w.H), dtype=torch.bfloat16, **pin)
     h2d = x_h.numel() * 2 + idx_h.numel() * 4 + w_h.numel() * 4 + (0 if eo_h is None else eo_h.numel() * 2)
@@ -331,22 +360,22 @@ def run_gpu(args, rank, world):
         with torch.cuda.stream(stream):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            xd.copy_(x_h, non_blocking=True)
-            idd.copy_(idx_h, non_blocking=True)
-            wd.copy_(w_h, non_blocking=True)
+            st.x.copy_(x_h, non_blocking=True)
+            st.idx.copy_(idx_h, non_blocking=True)
+            st.w.copy_(w_h, non_blocking=True)
             if eo_h is not None:
-                eo.copy_(eo_h, non_blocking=True)
-            do_dispatch()
-            do_combine()
-            y_h.copy_(y, non_blocking=True)
+                st.eo.copy_(eo_h, non_blocking=True)
+            do_dispatch(st)
+            do_combine(st)
+            st.y_h = y_h.copy_(st.y, non_blocking=True)
             e1.record(stream)
         e1.synchronize()
         if i >= args.warmup:
             e2e_ms.append(e0.elapsed_time(e1))
 
-    return dict(w=w, buf=buf, disp_ms=disp_ms, comb_ms=comb_ms, step_ms=step_ms,
-                total_ms=total_ms, clocks=clocks, launches_per_step=launches_per_step,
-                e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, moe=moe)
+    return dict(w=w, total_ms=total_ms, disp_ms=disp_ms, comb_ms=comb_ms, clocks=clocks,
+                launches_per_step=launches_per_step, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h,
+                nsets=nsets, set_bytes=set_bytes, l2=l2)
 
 
 def main():
@@ -397,15 +426,15 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     r = run_gpu(args, rank, world)
-    w, moe = r["w"], r["moe"]
+    w = r["w"]
     db, cb = algorithmic_bytes(w.T, w.H, w.E, w.R, w.k, w.fp8)
     step_bytes = db + cb
     ms_per_step = r["total_ms"] / args.steps
     value = step_bytes * world / (ms_per_step * 1e-3) / 1e9
 
-    disp_us = statistics.median(r["disp_ms"]) * 1e3
-    comb_us = statistics.median(r["comb_ms"]) * 1e3
-    comb_mean_s = statistics.mean(r["comb_ms"]) * 1e-3
+    disp_us = r["disp_ms"] / args.steps * 1e3
+    comb_us = r["comb_ms"] / args.steps * 1e3
+    comb_mean_s = comb_us * 1e-6
     ck_bytes = combine_kernel_bytes(w.T, w.H, w.k)
     achieved = ck_bytes / comb_mean_s / 1e9
     roofline = {"bound": "hbm", "kernel": "combine_rows", "achieved": round(achieved, 1),
@@ -422,7 +451,9 @@ def main():
         "config": {"workload": w.name, "T": w.T, "H": w.H, "E": w.E, "R": w.R, "k": w.k,
                    "payload": "fp8 e4m3 + fp32 scale per 128" if w.fp8 else "bf16",
                    "pad128": w.pad128, "combine": "bf16 out, fp32 accumulate",
-                   "l2": "flushed (2x L2 memset) before every step", "graphs": True,
+                   "l2": (f"inputs larger than L2: {r['nsets']} rotating sets of "
+                          f"{r['set_bytes'] / 1e6:.1f} MB (L2 {r['l2'] / 1e6:.0f} MB)"),
+                   "graphs": "one CUDA graph per step, replayed back to back",
                    "parallelism": f"replicas x{world}"},
         "dispatch_us": round(disp_us, 2), "combine_us": round(comb_us, 2),
         "total_us": round(ms_per_step * 1e3, 2),

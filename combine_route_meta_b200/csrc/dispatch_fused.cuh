@@ -6,8 +6,8 @@
 // Combinação"), shaped for decode batches where one launch and one DRAM round
 // trip cost more than the bytes.
 //
-// One CTA per token t; its warps own the 512-column chunks of x[t] in the
-// scatter's layout.  The CTA first issues the loads of x[t] (they do not
+// One CTA per token t; its warps own 256-column chunks of x[t] (the scatter's
+// layout with 8 columns per lane, so a decode row gets up to 32 warps).  The CTA first issues the loads of x[t] (they do not
 // depend on the routing), then reads all S = T*k expert ids (a few KB, served
 // from L2 after the first CTA) and builds in shared memory the histogram of all
 // entries and, in the same pass, the histogram of the entries that come before
@@ -29,8 +29,9 @@ namespace moe {
 
 constexpr int kFusedMaxEntries = 2048;
 constexpr int kFusedMaxK = 16;
-constexpr int kFusedMaxThreads = 512;
-constexpr int kFusedMaxChunks = 4; // 512-column chunks per warp: rows up to 16 warps x 4 x 512
+constexpr int kFusedMaxThreads = 1024;
+constexpr int kFusedLaneCols = 8;   // 256-column chunks: twice the warps per row of the scatter
+constexpr int kFusedMaxChunks = 4;  // chunks per warp: rows up to 32 warps x 4 x 256 columns
 constexpr int kFusedLoadRounds = 4; // expert ids loaded together per thread
 
 struct FusedArgs {
@@ -48,7 +49,7 @@ struct FusedArgs {
 inline size_t fused_smem(int32_t E) { return sizeof(int32_t) * ((size_t)3 * E + 1); }
 
 template <int kChunks, bool kFp8>
-__global__ void __launch_bounds__(kFusedMaxThreads) dispatch_fused(FusedArgs a)
+__global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_fused(FusedArgs a)
 {
     extern __shared__ int32_t sm[];
     int32_t *hist = sm, *before = sm + a.E, *off = sm + 2 * a.E;
@@ -60,16 +61,17 @@ __global__ void __launch_bounds__(kFusedMaxThreads) dispatch_fused(FusedArgs a)
     const int nwarps = nt / kWarp;
     const int warp = threadIdx.x / kWarp;
     const unsigned lane = lane_id();
-    const int32_t chunks = (a.H + kChunkCols - 1) / kChunkCols;
+    constexpr int L = kFusedLaneCols;
+    const int32_t chunks = (a.H + chunk_cols<L>() - 1) / chunk_cols<L>();
 
     // 1. The row's loads go out first: warp w owns chunks w, w + nwarps, ...
     const uint16_t *xr = a.x + (int64_t)t * a.H;
-    uint4 v0[kChunks], v1[kChunks];
+    LaneData<L> d[kChunks];
 #pragma unroll
     for (int i = 0; i < kChunks; ++i) {
         const int32_t c = warp + i * nwarps;
         if (c < chunks)
-            load_chunk<kFp8>(xr, a.H, c, v0[i], v1[i]);
+            load_chunk<L, kFp8>(xr, a.H, c, d[i]);
     }
 
     // 2. Histograms of all entries and of the entries before token t; the
@@ -152,7 +154,7 @@ __global__ void __launch_bounds__(kFusedMaxThreads) dispatch_fused(FusedArgs a)
     for (int i = 0; i < kChunks; ++i) {
         const int32_t c = warp + i * nwarps;
         if (c < chunks)
-            store_chunk<kFp8>(a.recv_x, a.recv_scale, a.H, c, a.k, s_slot, v0[i], v1[i]);
+            store_chunk<L, kFp8>(a.recv_x, a.recv_scale, a.H, c, a.k, s_slot, d[i]);
     }
 }
 

@@ -84,7 +84,7 @@ bool use_single_block(int64_t S) { return S <= kSingleBlockEntries; }
 int fused_chunks(const moe_config *c, int32_t T, unsigned *threads)
 {
     const int64_t S = (int64_t)T * c->k;
-    const int32_t chunks = (c->H + kChunkCols - 1) / kChunkCols;
+    const int32_t chunks = (c->H + chunk_cols<kFusedLaneCols>() - 1) / chunk_cols<kFusedLaneCols>();
     if (T <= 0 || S > kFusedMaxEntries || c->k > kFusedMaxK)
         return 0;
     const int max_warps = kFusedMaxThreads / kWarp;
@@ -301,7 +301,8 @@ int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
         a.k = cfg->k;
         a.recv_x = out->recv_x;
         a.recv_scale = out->recv_scale;
-        const int64_t warp_units = (int64_t)T * ((cfg->H + kChunkCols - 1) / kChunkCols);
+        constexpr int kCols = chunk_cols<kScatterLaneCols>();
+        const int64_t warp_units = (int64_t)T * ((cfg->H + kCols - 1) / kCols);
         const int warps_per_cta = kScatterThreads / kWarp;
         const unsigned grid =
             grid_for((warp_units + warps_per_cta - 1) / warps_per_cta, dev->sms, 2048 / kScatterThreads);
