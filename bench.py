@@ -251,7 +251,7 @@ def run_gpu(args, rank, world):
     recv_bytes = rows_cap * w.H * (1 if w.fp8 else 2) + (rows_cap * (w.H // 128) * 4 if w.fp8 else 0)
     set_bytes = (x.nbytes + idx.nbytes + wts.nbytes + (0 if eo_host is None else eo_host.nbytes)
                  + recv_bytes + rows_cap * 4 + idx.nbytes + w.T * w.H * 2)
-    nsets = 1 if set_bytes >= 2 * l2 else math.ceil(2 * l2 / set_bytes) + 1
+    nsets = 1 if set_bytes >= 2 * l2 else min(64, math.ceil(2 * l2 / set_bytes) + 1)
 
     class Set:
         pass
@@ -451,8 +451,9 @@ def main():
         "config": {"workload": w.name, "T": w.T, "H": w.H, "E": w.E, "R": w.R, "k": w.k,
                    "payload": "fp8 e4m3 + fp32 scale per 128" if w.fp8 else "bf16",
                    "pad128": w.pad128, "combine": "bf16 out, fp32 accumulate",
-                   "l2": (f"inputs larger than L2: {r['nsets']} rotating sets of "
-                          f"{r['set_bytes'] / 1e6:.1f} MB (L2 {r['l2'] / 1e6:.0f} MB)"),
+                   "l2": (f"{r['nsets']} rotating sets of {r['set_bytes'] / 1e6:.1f} MB "
+                          f"({r['nsets'] * r['set_bytes'] / 1e6:.0f} MB touched between uses of a "
+                          f"set; L2 {r['l2'] / 1e6:.0f} MB)"),
                    "graphs": "one CUDA graph per step, replayed back to back",
                    "parallelism": f"replicas x{world}"},
         "dispatch_us": round(disp_us, 2), "combine_us": round(comb_us, 2),
