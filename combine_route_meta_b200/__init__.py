@@ -42,6 +42,7 @@ ERR_INVALID_ARG = -1
 ERR_UNSUPPORTED = -2
 ERR_CUDA = -3
 ERR_DEVICE = -4
+ERR_TOO_LARGE = -5
 
 DEV_BAD_INDEX = 1
 DEV_CAPACITY = 2
@@ -50,6 +51,7 @@ DEV_BAD_SLOT = 8
 
 MAX_EXPERTS = 2048
 MAX_TOPK = 64
+NO_ALLOC_SCRATCH_BYTES = 1 << 20
 
 
 class moe_config(ctypes.Structure):
@@ -87,6 +89,9 @@ def _declare(lib):
     lib.moe_dispatch.argtypes = [cfgp, i32, P, P, P, ctypes.POINTER(moe_dispatch_out), P, P,
                                  ctypes.c_size_t, P, P, ctypes.POINTER(moe_handle)]
     lib.moe_dispatch.restype = ctypes.c_int
+    lib.moe_dispatch_no_alloc.argtypes = [cfgp, i32, P, P, P, ctypes.POINTER(moe_dispatch_out), P,
+                                          P, P, ctypes.POINTER(moe_handle)]
+    lib.moe_dispatch_no_alloc.restype = ctypes.c_int
     lib.moe_combine.argtypes = [ctypes.POINTER(moe_handle), P, P, P, P]
     lib.moe_combine.restype = ctypes.c_int
     lib.moe_check.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
@@ -103,6 +108,7 @@ moe_rows_capacity = lib.moe_rows_capacity
 moe_workspace_bytes = lib.moe_workspace_bytes
 moe_dispatch_sizes_for = lib.moe_dispatch_sizes_for
 moe_dispatch = lib.moe_dispatch
+moe_dispatch_no_alloc = lib.moe_dispatch_no_alloc
 moe_combine = lib.moe_combine
 moe_check = lib.moe_check
 

@@ -3,6 +3,7 @@
 // include/moe_dispatch_combine.h.
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include <cuda_runtime.h>
 
@@ -13,6 +14,12 @@
 #include "dispatch_fused.cuh"
 #include "meta.cuh"
 #include "scatter.cuh"
+
+// Scratch of moe_dispatch_no_alloc: a fixed array in device memory, allocated
+// by the CUDA runtime when the library's module is loaded on a device and held
+// there until the process exits.  Host code must not use this name as a device
+// address; it resolves the address with cudaGetSymbolAddress (below).
+static __device__ __align__(256) int32_t g_no_alloc_scratch[MOE_NO_ALLOC_SCRATCH_BYTES / sizeof(int32_t)];
 
 namespace moe {
 namespace {
@@ -45,6 +52,27 @@ int device_info(DeviceInfo **out)
         d.ready = true;
     }
     *out = &d;
+    return MOE_OK;
+}
+
+// Device address of g_no_alloc_scratch on the current device, looked up once
+// per device (with that device current) and cached.
+void *g_no_alloc_addr[kMaxDevices];
+std::mutex g_no_alloc_mutex;
+
+int no_alloc_scratch(void **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_no_alloc_mutex);
+    if (g_no_alloc_addr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_no_alloc_scratch) != cudaSuccess || p == nullptr)
+            return MOE_ERR_CUDA;
+        g_no_alloc_addr[dev] = p;
+    }
+    *out = g_no_alloc_addr[dev];
     return MOE_OK;
 }
 
@@ -156,6 +184,8 @@ const char *moe_status_string(int status)
         return "CUDA error";
     case MOE_ERR_DEVICE:
         return "device reported an error";
+    case MOE_ERR_TOO_LARGE:
+        return "problem needs more scratch than the fixed no-allocation buffer holds";
     default:
         return "unknown status";
     }
@@ -357,6 +387,28 @@ int moe_combine(const moe_handle *handle, const void *expert_out, void *y, int32
     const unsigned grid = grid_for((int64_t)a.T * a.parts, dev->sms, 16);
     combine_rows<<<grid, kCombineThreads, 0, static_cast<cudaStream_t>(stream)>>>(a);
     return launched(cudaGetLastError());
+}
+
+int moe_dispatch_no_alloc(const moe_config *cfg, int32_t T, const void *x,
+                          const int32_t *topk_idx, const float *topk_w,
+                          const moe_dispatch_out *out, int32_t *slot, int32_t *dev_err,
+                          void *stream, moe_handle *handle)
+{
+    int st = check_config(cfg);
+    if (st != MOE_OK)
+        return st;
+    if (T < 0)
+        return MOE_ERR_INVALID_ARG;
+    const size_t need = workspace_bytes(cfg, T);
+    if (need > MOE_NO_ALLOC_SCRATCH_BYTES)
+        return MOE_ERR_TOO_LARGE;
+    void *scratch = nullptr;
+    if ((st = no_alloc_scratch(&scratch)) != MOE_OK)
+        return st;
+    // The tiled metadata kernels write every scratch word they later read, so
+    // the array needs no clearing between calls.
+    return moe_dispatch(cfg, T, x, topk_idx, topk_w, out, slot, need > 0 ? scratch : nullptr, need,
+                        dev_err, stream, handle);
 }
 
 int moe_check(int32_t *dev_err, void *stream, int32_t *bits_out)

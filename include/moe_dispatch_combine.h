@@ -65,6 +65,7 @@ extern "C" {
 #define MOE_ERR_UNSUPPORTED -2 /* a valid request outside what the kernels cover */
 #define MOE_ERR_CUDA -3        /* a CUDA runtime call or launch failed            */
 #define MOE_ERR_DEVICE -4      /* moe_check: the device error word was non-zero  */
+#define MOE_ERR_TOO_LARGE -5   /* moe_dispatch_no_alloc: scratch would not fit    */
 
 /* Bits of the device error word. */
 #define MOE_DEV_BAD_INDEX 1 /* dispatch: an expert id outside [0, E)                  */
@@ -75,6 +76,7 @@ extern "C" {
 /* Limits of this build. */
 #define MOE_MAX_EXPERTS 2048 /* E */
 #define MOE_MAX_TOPK 64      /* k */
+#define MOE_NO_ALLOC_SCRATCH_BYTES (1u << 20) /* fixed scratch of moe_dispatch_no_alloc */
 
 /*
  * Problem description.
@@ -197,6 +199,36 @@ MOE_API int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const 
  */
 MOE_API int moe_combine(const moe_handle *handle, const void *expert_out, void *y, int32_t *dev_err,
                 void *stream);
+
+/*
+ * moe_dispatch without a workspace argument, for callers that cannot allocate
+ * device memory (the pages have no counterpart; this is a deployment aid).
+ *
+ * Some callers may not call cudaMalloc or any allocator: code that runs while
+ * a stream is being captured into a CUDA graph, serving loops with a memory
+ * plan fixed at start-up, and plain C hosts that are only handed device
+ * pointers.  This entry point takes the same inputs and caller-allocated
+ * outputs as moe_dispatch and computes the same results, but its metadata
+ * scratch is a fixed MOE_NO_ALLOC_SCRATCH_BYTES array inside the library
+ * (device memory that every GPU which loads the library holds until the
+ * process exits).  It allocates nothing and frees nothing.
+ *
+ * - Limit: the tiled metadata needs ceil(T*k/1024) * E int32 words
+ *   (moe_workspace_bytes); beyond MOE_NO_ALLOC_SCRATCH_BYTES the call returns
+ *   MOE_ERR_TOO_LARGE and enqueues nothing.  With E = 256 that allows T*k up
+ *   to 1,048,576 entries; with E = 2048, up to 131,072.
+ * - Set-up: the first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current.  Make that first call
+ *   before capturing any stream.
+ * - Sharing: every call on a device uses the same array and leaves its
+ *   contents behind; the kernels overwrite every word they read, so nothing
+ *   needs clearing.  Calls whose work overlaps on the GPU (different streams
+ *   with no ordering between them) race on the array and must not be made.
+ */
+MOE_API int moe_dispatch_no_alloc(const moe_config *cfg, int32_t T, const void *x,
+                                  const int32_t *topk_idx, const float *topk_w,
+                                  const moe_dispatch_out *out, int32_t *slot, int32_t *dev_err,
+                                  void *stream, moe_handle *handle);
 
 /*
  * Waits for `stream`, reads the device error word, clears it (stream-ordered),
