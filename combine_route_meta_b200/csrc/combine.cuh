@@ -37,6 +37,7 @@ struct CombineArgs {
 
 __global__ void __launch_bounds__(kCombineThreads) combine_rows(CombineArgs a)
 {
+    stream_order_begin();
     const int32_t nvec = a.H / 8;
     const int64_t units = (int64_t)a.T * a.parts;
     for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {

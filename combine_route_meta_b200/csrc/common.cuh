@@ -19,6 +19,18 @@ __device__ __forceinline__ void raise_error(int32_t *err, int32_t bit)
 
 __device__ __forceinline__ unsigned lane_id() { return threadIdx.x & (kWarp - 1); }
 
+// Programmatic dependent launch.  Every kernel here is launched so that it may
+// start while the previous kernel in the stream is still finishing.  Before its
+// first global-memory access it waits for that kernel to complete and its
+// writes to be visible (so stream order still holds for every buffer), then
+// lets the next kernel start launching.  The next kernel's launch therefore
+// overlaps this one's tail; the wait itself is done by the hardware.
+__device__ __forceinline__ void stream_order_begin()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ unsigned lanemask_lt()
 {
     unsigned m;

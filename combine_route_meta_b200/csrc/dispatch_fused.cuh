@@ -51,6 +51,7 @@ inline size_t fused_smem(int32_t E) { return sizeof(int32_t) * ((size_t)3 * E + 
 template <int kChunks, bool kFp8>
 __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_fused(FusedArgs a)
 {
+    stream_order_begin();
     extern __shared__ int32_t sm[];
     int32_t *hist = sm, *before = sm + a.E, *off = sm + 2 * a.E;
     __shared__ int32_t s_slot[kFusedMaxK];

@@ -242,6 +242,7 @@ constexpr int kSingleRounds = kSingleBlockEntries / kMetaThreads;
 // Shared memory: cnt[E], off[E+1], cursor[E], wcnt[kMetaWarps*E].
 __global__ void __launch_bounds__(kMetaThreads) meta_single_block(MetaArgs a)
 {
+    stream_order_begin();
     extern __shared__ int32_t sm[];
     int32_t *cnt = sm, *off = sm + a.E, *cursor = off + a.E + 1, *wcnt = cursor + a.E;
     for (int32_t e = threadIdx.x; e < a.E; e += kMetaThreads)
@@ -266,6 +267,7 @@ constexpr int kTileRounds = kTileEntries / kMetaThreads;
 // (1) tile_hist[tile][e] = entries of tile `tile` routed to e.
 __global__ void __launch_bounds__(kMetaThreads) meta_tile_count(MetaArgs a, int32_t *tile_hist)
 {
+    stream_order_begin();
     extern __shared__ int32_t hist[];
     for (int32_t e = threadIdx.x; e < a.E; e += kMetaThreads)
         hist[e] = 0;
@@ -288,6 +290,7 @@ constexpr int kScanWarps = kScanThreads / kWarp;
 __global__ void __launch_bounds__(kScanThreads) meta_tile_scan(MetaArgs a, int32_t *tile_hist,
                                                                int32_t ntiles)
 {
+    stream_order_begin();
     __shared__ int32_t part[kScanWarps][kWarp];
     const int warp = threadIdx.x / kWarp, lane = lane_id();
     const int32_t e = blockIdx.x * kWarp + lane;
@@ -337,6 +340,7 @@ __global__ void __launch_bounds__(kScanThreads) meta_tile_scan(MetaArgs a, int32
 __global__ void __launch_bounds__(kMetaThreads) meta_tile_assign(MetaArgs a,
                                                                  const int32_t *tile_prefix)
 {
+    stream_order_begin();
     extern __shared__ int32_t sm[];
     int32_t *cnt = sm, *off = sm + a.E, *cursor = off + a.E + 1, *wcnt = cursor + a.E;
     for (int32_t e = threadIdx.x; e < a.E; e += kMetaThreads) {

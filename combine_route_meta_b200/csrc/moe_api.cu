@@ -78,6 +78,26 @@ int no_alloc_scratch(void **out)
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Launches a kernel that may begin while the previous kernel in the stream is
+// finishing (programmatic stream serialization); each kernel starts with
+// stream_order_begin(), which waits for that kernel before touching memory.
+template <typename... Params, typename... Args>
+cudaError_t launch(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                   Args... args)
+{
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 int check_config(const moe_config *c)
 {
     if (c == nullptr)
@@ -130,16 +150,12 @@ cudaError_t launch_fused(int per, unsigned grid, unsigned block, size_t smem, cu
 {
     switch (per) {
     case 1:
-        dispatch_fused<1, kFp8><<<grid, block, smem, s>>>(f);
-        break;
+        return launch(dispatch_fused<1, kFp8>, grid, block, smem, s, f);
     case 2:
-        dispatch_fused<2, kFp8><<<grid, block, smem, s>>>(f);
-        break;
+        return launch(dispatch_fused<2, kFp8>, grid, block, smem, s, f);
     default:
-        dispatch_fused<4, kFp8><<<grid, block, smem, s>>>(f);
-        break;
+        return launch(dispatch_fused<4, kFp8>, grid, block, smem, s, f);
     }
-    return cudaGetLastError();
 }
 
 size_t workspace_bytes(const moe_config *c, int32_t T)
@@ -308,17 +324,19 @@ int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
     }
 
     if (use_single_block(S)) {
-        meta_single_block<<<1, kMetaThreads, meta_single_smem(cfg->E), s>>>(m);
-        if ((st = launched(cudaGetLastError())) != MOE_OK)
+        if ((st = launched(launch(meta_single_block, 1, kMetaThreads, meta_single_smem(cfg->E), s,
+                                  m))) != MOE_OK)
             return st;
     } else {
         const int64_t ntiles = meta_tiles(S);
         int32_t *tile_hist = static_cast<int32_t *>(workspace);
-        meta_tile_count<<<(unsigned)ntiles, kMetaThreads, meta_count_smem(cfg->E), s>>>(m, tile_hist);
-        meta_tile_scan<<<(unsigned)((cfg->E + kWarp - 1) / kWarp), kScanThreads, 0, s>>>(
-            m, tile_hist, (int32_t)ntiles);
-        meta_tile_assign<<<(unsigned)ntiles, kMetaThreads, meta_assign_smem(cfg->E), s>>>(m, tile_hist);
-        if ((st = launched(cudaGetLastError())) != MOE_OK)
+        const int32_t *tile_prefix = tile_hist;
+        if ((st = launched(launch(meta_tile_count, (unsigned)ntiles, kMetaThreads,
+                                  meta_count_smem(cfg->E), s, m, tile_hist))) != MOE_OK ||
+            (st = launched(launch(meta_tile_scan, (unsigned)((cfg->E + kWarp - 1) / kWarp),
+                                  kScanThreads, 0, s, m, tile_hist, (int32_t)ntiles))) != MOE_OK ||
+            (st = launched(launch(meta_tile_assign, (unsigned)ntiles, kMetaThreads,
+                                  meta_assign_smem(cfg->E), s, m, tile_prefix))) != MOE_OK)
             return st;
     }
 
@@ -336,11 +354,9 @@ int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
         const int warps_per_cta = kScatterThreads / kWarp;
         const unsigned grid =
             grid_for((warp_units + warps_per_cta - 1) / warps_per_cta, dev->sms, 2048 / kScatterThreads);
-        if (fp8)
-            scatter_rows<true><<<grid, kScatterThreads, 0, s>>>(a);
-        else
-            scatter_rows<false><<<grid, kScatterThreads, 0, s>>>(a);
-        if ((st = launched(cudaGetLastError())) != MOE_OK)
+        const cudaError_t e = fp8 ? launch(scatter_rows<true>, grid, kScatterThreads, 0, s, a)
+                                  : launch(scatter_rows<false>, grid, kScatterThreads, 0, s, a);
+        if ((st = launched(e)) != MOE_OK)
             return st;
     }
 
@@ -385,8 +401,7 @@ int moe_combine(const moe_handle *handle, const void *expert_out, void *y, int32
     a.y = static_cast<uint16_t *>(y);
     a.err = dev_err;
     const unsigned grid = grid_for((int64_t)a.T * a.parts, dev->sms, 16);
-    combine_rows<<<grid, kCombineThreads, 0, static_cast<cudaStream_t>(stream)>>>(a);
-    return launched(cudaGetLastError());
+    return launched(launch(combine_rows, grid, kCombineThreads, 0, static_cast<cudaStream_t>(stream), a));
 }
 
 int moe_dispatch_no_alloc(const moe_config *cfg, int32_t T, const void *x,

@@ -17,9 +17,9 @@
 //  - bf16: lane l moves the 16-byte vectors at columns 8l (+ 256 when L = 16);
 //  - fp8: lane l owns L consecutive columns, 128/L lanes make one 128-column
 //    block; the block's |x| maximum is reduced with butterfly shuffles inside
-//    those lanes, the scale is amax/448 and each code is e4m3(x/scale) (IEEE
-//    round-to-nearest divisions, saturating round-to-nearest-even
-//    conversion).  A lane stores its L codes with one L-byte store, and lane 0
+//    those lanes, the scale is amax/448 and each code is e4m3(x/scale) with
+//    the binary32 quotient correctly rounded (see quotient_for_e4m3) and a
+//    saturating round-to-nearest-even conversion.  A lane stores its L codes with one L-byte store, and lane 0
 //    stores the warp's L/4 block scales with one store when the scale row
 //    allows it.
 // The token's k slots are read once per unit (lane j holds slot j) and
@@ -49,6 +49,29 @@ template <int kLaneCols>
 struct LaneData {
     uint4 v[kLaneCols / 8];
 };
+
+// x / scale as the e4m3 conversion needs it.  The codes must equal those of the
+// correctly rounded binary32 quotient.  With recip = RN(1/scale), the product
+// q = RN(x * recip) lies within 2.5 units in the last place of RN(x / scale)
+// (two relative roundings of 2^-24 each, plus the half unit of RN itself).
+// e4m3 rounding is monotone and its rounding boundaries in the normal range
+// are the values whose 20 low mantissa bits are exactly 0x80000 (halfway
+// between two 3-bit mantissas).  So when q is in the e4m3 normal range
+// (>= 2^-6) and more than 3 units from such a boundary, both quotients give
+// the same code and q is used; otherwise (near a boundary, in the e4m3
+// subnormal range, a zero, or a block whose scale is below FLT_MIN) the exact
+// division is taken.  On N(0,1) data the slow branch is rare (~1e-4).
+__device__ __forceinline__ float quotient_for_e4m3(float x, float scale, float recip, bool fast)
+{
+    if (fast) {
+        const float q = x * recip;
+        const uint32_t b = __float_as_uint(q) & 0x7fffffffu;
+        const int32_t off_mid = (int32_t)(b & 0xfffffu) - 0x80000;
+        if (b >= 0x3c800000u && (off_mid > 3 || off_mid < -3))
+            return q;
+    }
+    return __fdiv_rn(x, scale);
+}
 
 // e4m3 codes of the lane's values, element 0 in the lowest byte, and the scale
 // of the lane's 128-column block.  All lanes of the warp call this together
@@ -83,10 +106,14 @@ __device__ __forceinline__ void quantise_lane(const LaneData<kLaneCols> &d, uint
         codes[i] = 0u;
     if (amax > 0.0f) {
         scale = __fdiv_rn(amax, 448.0f);
+        const float recip = __frcp_rn(scale);
+        const bool fast = scale >= 0x1p-126f; // recip finite, products in range
 #pragma unroll
         for (int i = 0; i < kLaneCols / 4; ++i) {
-            const float q0 = __fdiv_rn(f[4 * i + 0], scale), q1 = __fdiv_rn(f[4 * i + 1], scale);
-            const float q2 = __fdiv_rn(f[4 * i + 2], scale), q3 = __fdiv_rn(f[4 * i + 3], scale);
+            const float q0 = quotient_for_e4m3(f[4 * i + 0], scale, recip, fast);
+            const float q1 = quotient_for_e4m3(f[4 * i + 1], scale, recip, fast);
+            const float q2 = quotient_for_e4m3(f[4 * i + 2], scale, recip, fast);
+            const float q3 = quotient_for_e4m3(f[4 * i + 3], scale, recip, fast);
             codes[i] = pack_e4m3x2(q0, q1) | (pack_e4m3x2(q2, q3) << 16);
         }
     }
@@ -192,6 +219,7 @@ __device__ __forceinline__ void store_chunk(void *recv_x, float *recv_scale, int
 template <bool kFp8>
 __global__ void __launch_bounds__(kScatterThreads) scatter_rows(ScatterArgs a)
 {
+    stream_order_begin();
     constexpr int L = kScatterLaneCols;
     const int64_t nwarps = (int64_t)gridDim.x * (kScatterThreads / kWarp);
     const int32_t chunks = (a.H + chunk_cols<L>() - 1) / chunk_cols<L>();

@@ -323,3 +323,47 @@ def test_torch_level_api():
     o = oracle.dispatch(x, idx, E=w.E, R=w.R, fp8=False)
     np.testing.assert_array_equal(d.expert_offset.cpu().numpy(), o["expert_offset"])
     assert_combine_close(bf16_from_dev(y), oracle.combine(o["slot"], wts, o["recv_x"]))
+
+
+def _all_bf16_blocks(rng):
+    """Rows of 128-column blocks: each block starts with its amax A and then walks through
+    every bf16 value of magnitude <= A (both signs), for about 30 amax values A."""
+    amaxes = [0x0040, 0x0080, 0x0101, 0x1F35, 0x2F00, 0x3A8F, 0x3B80, 0x3C00, 0x3D4D, 0x3E80,
+              0x3F00, 0x3F80, 0x3FC9, 0x4000, 0x4049, 0x40A0, 0x4120, 0x41A0, 0x4300, 0x43E0,
+              0x4400, 0x4500, 0x4680, 0x4780, 0x4B00, 0x5000, 0x5A5A, 0x6000, 0x7000, 0x7F7F]
+    blocks = []
+    for a in amaxes:
+        vals = np.arange(0, a + 1, dtype=np.uint32)
+        vals = np.concatenate([vals, vals | 0x8000]).astype(np.uint16)
+        rng.shuffle(vals)
+        n = (len(vals) + 126) // 127
+        vals = np.resize(vals, n * 127)
+        blk = np.empty((n, 128), np.uint16)
+        blk[:, 0] = a if rng.random() < 0.5 else a | 0x8000
+        blk[:, 1:] = vals.reshape(n, 127)
+        blocks.append(blk)
+    blocks = np.concatenate(blocks)
+    per_row = 64
+    rows = (len(blocks) + per_row - 1) // per_row
+    blocks = np.resize(blocks, (rows * per_row, 128))
+    return blocks.reshape(rows, per_row * 128)
+
+
+@pytest.mark.parametrize("k", [1, 17], ids=["fused", "scatter"])
+def test_fp8_quantiser_every_bf16_value(k):
+    # every bf16 magnitude below each block's amax, through the kernel's quotient shortcut and
+    # its exact fallback; codes and scales must equal the oracle's bit for bit
+    rng = np.random.default_rng(2024)
+    x = _all_bf16_blocks(rng)
+    T = x.shape[0]
+    idx = np.tile(np.arange(k, dtype=np.int32), (T, 1))
+    w = np.full((T, k), 1.0 / k, np.float32)
+    buf, bits, _ = run_gpu(x, idx, w, E=k, R=1, fp8=True)
+    assert bits == 0
+    g = dispatch_host(buf)
+    for t in range(T):
+        codes, scales = oracle.quantise_row_fp8(x[t])
+        for j in (0, k - 1):
+            s = g["slot"][t, j]
+            np.testing.assert_array_equal(g["recv_x"][s], codes, err_msg=f"row {t}")
+            np.testing.assert_array_equal(g["recv_scale"][s].view(np.uint32), scales.view(np.uint32))
