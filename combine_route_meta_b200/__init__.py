@@ -94,6 +94,8 @@ def _declare(lib):
     lib.moe_dispatch_no_alloc.restype = ctypes.c_int
     lib.moe_combine.argtypes = [ctypes.POINTER(moe_handle), P, P, P, P]
     lib.moe_combine.restype = ctypes.c_int
+    lib.moe_selftest_bounded_wait.argtypes = [P, ctypes.c_uint64, P]
+    lib.moe_selftest_bounded_wait.restype = ctypes.c_int
     lib.moe_check.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
     lib.moe_check.restype = ctypes.c_int
     return lib
@@ -111,6 +113,7 @@ moe_dispatch = lib.moe_dispatch
 moe_dispatch_no_alloc = lib.moe_dispatch_no_alloc
 moe_combine = lib.moe_combine
 moe_check = lib.moe_check
+moe_selftest_bounded_wait = lib.moe_selftest_bounded_wait
 
 
 class MoeError(RuntimeError):

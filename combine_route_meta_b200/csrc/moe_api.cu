@@ -22,6 +22,22 @@
 static __device__ __align__(256) int32_t g_no_alloc_scratch[MOE_NO_ALLOC_SCRATCH_BYTES / sizeof(int32_t)];
 
 namespace moe {
+
+// Diagnostic: waits on an mbarrier that nothing completes, with the same bounded
+// wait the bulk kernels use, and reports MOE_DEV_TIMEOUT when it gives up.
+__global__ void __launch_bounds__(kWarp) wait_selftest(int32_t *err, uint64_t limit_ns)
+{
+    stream_order_begin();
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_addr(&bar), 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    if (threadIdx.x == 0 && !mbar_wait(smem_addr(&bar), 0, limit_ns))
+        raise_error(err, MOE_DEV_TIMEOUT);
+}
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -47,7 +63,9 @@ int device_info(DeviceInfo **out)
         if (cudaFuncSetAttribute(meta_single_block, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)big) != cudaSuccess ||
             cudaFuncSetAttribute(meta_tile_assign, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)meta_assign_smem(MOE_MAX_EXPERTS)) != cudaSuccess)
+                                 (int)meta_assign_smem(MOE_MAX_EXPERTS)) != cudaSuccess ||
+            cudaFuncSetAttribute(scatter_bulk_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kBulkMaxSmem) != cudaSuccess)
             return MOE_ERR_CUDA;
         d.ready = true;
     }
@@ -349,13 +367,20 @@ int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
         a.k = cfg->k;
         a.recv_x = out->recv_x;
         a.recv_scale = out->recv_scale;
-        constexpr int kCols = chunk_cols<kScatterLaneCols>();
-        const int64_t warp_units = (int64_t)T * ((cfg->H + kCols - 1) / kCols);
-        const int warps_per_cta = kScatterThreads / kWarp;
-        const unsigned grid =
-            grid_for((warp_units + warps_per_cta - 1) / warps_per_cta, dev->sms, 2048 / kScatterThreads);
-        const cudaError_t e = fp8 ? launch(scatter_rows<true>, grid, kScatterThreads, 0, s, a)
-                                  : launch(scatter_rows<false>, grid, kScatterThreads, 0, s, a);
+        cudaError_t e;
+        if (use_bulk_scatter(cfg->H, fp8)) {
+            const unsigned grid = grid_for(T, dev->sms, kBulkCtasPerSm);
+            const size_t smem = (size_t)kBulkStages * bulk_stage_bytes(cfg->H);
+            e = launch(scatter_bulk_bf16, grid, kWarp, smem, s, a, dev_err);
+        } else {
+            constexpr int kCols = chunk_cols<kScatterLaneCols>();
+            const int64_t warp_units = (int64_t)T * ((cfg->H + kCols - 1) / kCols);
+            const int warps_per_cta = kScatterThreads / kWarp;
+            const unsigned grid = grid_for((warp_units + warps_per_cta - 1) / warps_per_cta, dev->sms,
+                                           2048 / kScatterThreads);
+            e = fp8 ? launch(scatter_rows<true>, grid, kScatterThreads, 0, s, a)
+                    : launch(scatter_rows<false>, grid, kScatterThreads, 0, s, a);
+        }
         if ((st = launched(e)) != MOE_OK)
             return st;
     }
@@ -424,6 +449,14 @@ int moe_dispatch_no_alloc(const moe_config *cfg, int32_t T, const void *x,
     // the array needs no clearing between calls.
     return moe_dispatch(cfg, T, x, topk_idx, topk_w, out, slot, need > 0 ? scratch : nullptr, need,
                         dev_err, stream, handle);
+}
+
+int moe_selftest_bounded_wait(int32_t *dev_err, uint64_t limit_ns, void *stream)
+{
+    if (dev_err == nullptr || limit_ns == 0 || limit_ns > kWaitLimitNs)
+        return MOE_ERR_INVALID_ARG;
+    return launched(launch(wait_selftest, 1, kWarp, 0, static_cast<cudaStream_t>(stream), dev_err,
+                           limit_ns));
 }
 
 int moe_check(int32_t *dev_err, void *stream, int32_t *bits_out)

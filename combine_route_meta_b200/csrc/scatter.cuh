@@ -234,4 +234,88 @@ __global__ void __launch_bounds__(kScatterThreads) scatter_rows(ScatterArgs a)
     }
 }
 
+
+// ---- bulk (TMA) scatter, bf16 ------------------------------------------------------
+// The same results as scatter_rows<false>, for rows of at least 1 KB.  Each CTA
+// is one warp that walks tokens t = blockIdx.x, + gridDim.x, ... through a ring
+// of kBulkStages shared-memory stages:
+//   - lane 0 brings x[t] into a stage with one bulk copy (completion counted on
+//     the stage's mbarrier), kBulkLookahead tokens ahead;
+//   - lane j issues the bulk store of the row to slot j, so each receive row is
+//     written as one contiguous multi-kilobyte stream.
+// A stage is reloaded only after this warp's stores from it have finished
+// reading it.  Long contiguous writes per destination keep the HBM write stream
+// efficient, which is what bounds dispatch (k writes per read); many one-warp
+// CTAs run in waves, which balances the tail.
+constexpr int kBulkStages = 4;
+constexpr int kBulkLookahead = 2;
+constexpr int kBulkCtasPerSm = 16;
+constexpr uint32_t kBulkMaxSmem = 200 * 1024;
+
+__host__ __device__ inline uint32_t bulk_stage_bytes(int32_t H)
+{
+    return ((uint32_t)H * 2 + 127) / 128 * 128;
+}
+
+__global__ void __launch_bounds__(kWarp) scatter_bulk_bf16(ScatterArgs a, int32_t *err)
+{
+    stream_order_begin();
+    extern __shared__ __align__(128) uint8_t stage_mem[];
+    __shared__ __align__(8) uint64_t bars[kBulkStages];
+    const unsigned lane = lane_id();
+    const uint32_t row = (uint32_t)a.H * 2;
+    const uint32_t stage_bytes = bulk_stage_bytes(a.H);
+    if (lane == 0) {
+        for (int s = 0; s < kBulkStages; ++s)
+            mbar_init(smem_addr(&bars[s]), 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+
+    const int64_t n = ((int64_t)a.T - blockIdx.x + gridDim.x - 1) / gridDim.x;
+    auto token = [&](int64_t i) { return (int32_t)(blockIdx.x + i * gridDim.x); };
+    auto issue_load = [&](int64_t i) {
+        if (lane == 0) {
+            const int s = (int)(i % kBulkStages);
+            const uint32_t bar = smem_addr(&bars[s]);
+            mbar_expect_tx(bar, row);
+            bulk_load(smem_addr(stage_mem + s * stage_bytes), a.x + (int64_t)token(i) * a.H, row, bar);
+        }
+    };
+    for (int64_t i = 0; i < kBulkLookahead && i < n; ++i)
+        issue_load(i);
+
+    for (int64_t i = 0; i < n; ++i) {
+        const int s = (int)(i % kBulkStages);
+        if (!mbar_wait(smem_addr(&bars[s]), (uint32_t)((i / kBulkStages) & 1), kWaitLimitNs)) {
+            if (lane == 0)
+                raise_error(err, MOE_DEV_TIMEOUT);
+            break;
+        }
+        const int32_t t = token(i);
+        for (int32_t j = (int32_t)lane; j < a.k; j += kWarp) {
+            const int32_t d = __ldg(a.slot + (int64_t)t * a.k + j);
+            if (d >= 0)
+                bulk_store(static_cast<uint16_t *>(a.recv_x) + (int64_t)d * a.H,
+                           smem_addr(stage_mem + s * stage_bytes), row);
+        }
+        bulk_commit();
+        const int64_t next = i + kBulkLookahead;
+        if (next < n) {
+            bulk_wait_read<kBulkStages - kBulkLookahead>();
+            __syncwarp();
+            issue_load(next);
+        }
+    }
+    bulk_wait_all();
+}
+
+// Whether the bulk scatter applies: bf16 rows of at least 1 KB whose stages fit.
+// (fp8 stays on scatter_rows: its quantiser needs many warps per SM, and a
+// per-token barrier before the bulk stores cost more than they saved.)
+inline bool use_bulk_scatter(int32_t H, bool fp8)
+{
+    return !fp8 && H >= 512 && (uint64_t)kBulkStages * bulk_stage_bytes(H) <= kBulkMaxSmem;
+}
+
 } // namespace moe

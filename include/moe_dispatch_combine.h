@@ -70,7 +70,7 @@ extern "C" {
 /* Bits of the device error word. */
 #define MOE_DEV_BAD_INDEX 1 /* dispatch: an expert id outside [0, E)                  */
 #define MOE_DEV_CAPACITY 2  /* dispatch: a receive row at or past rows_cap            */
-#define MOE_DEV_TIMEOUT 4   /* a bounded device wait gave up                          */
+#define MOE_DEV_TIMEOUT 4   /* a bounded device wait (1 s) gave up                     */
 #define MOE_DEV_BAD_SLOT 8  /* combine: a slot outside [-1, rows_cap) in the handle   */
 
 /* Limits of this build. */
@@ -229,6 +229,17 @@ MOE_API int moe_dispatch_no_alloc(const moe_config *cfg, int32_t T, const void *
                                   const int32_t *topk_idx, const float *topk_w,
                                   const moe_dispatch_out *out, int32_t *slot, int32_t *dev_err,
                                   void *stream, moe_handle *handle);
+
+/*
+ * Diagnostic of the library's bounded device waits.  Launches one warp that
+ * waits on a shared-memory barrier nothing ever completes, using the same wait
+ * as the bulk-copy kernels, and gives up after limit_ns nanoseconds
+ * (1..1e9); it then ORs MOE_DEV_TIMEOUT into *dev_err (device pointer) and
+ * returns, leaving the context usable.  Every wait in the dispatch kernels has
+ * a 1 s limit and reports the same bit.  Returns a status; the bit is read with
+ * moe_check.
+ */
+MOE_API int moe_selftest_bounded_wait(int32_t *dev_err, uint64_t limit_ns, void *stream);
 
 /*
  * Waits for `stream`, reads the device error word, clears it (stream-ordered),

@@ -110,3 +110,10 @@ def test_sizes_for_fp8():
     assert moe.moe_dispatch_sizes_for(ctypes.byref(cfg), 128, 1024, ctypes.byref(s)) == moe.OK
     assert s.recv_x == 1024 * 7168 and s.recv_scale == 1024 * 56 * 4
     assert s.expert_offset == 257 * 4 and s.rank_offset == 9 * 4 and s.slot == 128 * 8 * 4
+
+
+def test_selftest_wait_rejects_bad_limits():
+    P = ctypes.c_void_p
+    assert moe.moe_selftest_bounded_wait(None, 1000, None) == moe.ERR_INVALID_ARG
+    assert moe.moe_selftest_bounded_wait(P(16), 0, None) == moe.ERR_INVALID_ARG
+    assert moe.moe_selftest_bounded_wait(P(16), 2_000_000_000, None) == moe.ERR_INVALID_ARG

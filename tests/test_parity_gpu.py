@@ -6,6 +6,8 @@ and scales) must match bit for bit.  Combine must satisfy, per element,
 are filled with a poison byte before the call, on both sides, so rows that
 must stay unwritten (padding, unused capacity) are compared too.
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -170,6 +172,7 @@ CASES = [
     (10, 128, 8, 2, 20, False, False, False),
     (600, 1032, 16, 4, 5, False, True, False),   # ragged last 512-column chunk (8 columns)
     (300, 1152, 8, 8, 8, True, True, True),      # 9 scales per row: no 16-byte scale stores
+    (3, 30720, 8, 2, 20, True, False, False),    # rows too wide for the bulk stages: register scatter
     (1, 128, 4, 2, 4, True, False, True),
     (5, 136, 6, 3, 3, False, False, True),       # H/8 = 17 vectors: one ragged part
     (33, 1032, 16, 4, 5, False, True, False),    # 129 vectors: two parts, duplicates
@@ -367,3 +370,16 @@ def test_fp8_quantiser_every_bf16_value(k):
             s = g["slot"][t, j]
             np.testing.assert_array_equal(g["recv_x"][s], codes, err_msg=f"row {t}")
             np.testing.assert_array_equal(g["recv_scale"][s].view(np.uint32), scales.view(np.uint32))
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    # a wait on a barrier nothing completes gives up after its limit and reports the bit
+    err = moe.error_word()
+    moe.check()
+    st = moe.moe_selftest_bounded_wait(ctypes.c_void_p(err.data_ptr()), 20_000_000,
+                                       ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == moe.OK
+    assert moe.check() == moe.DEV_TIMEOUT
+    # the context is still usable: a normal dispatch + combine matches the oracle
+    x, idx, w = random_problem(12, 64, 512, 8, 2)
+    check_problem(x, idx, w, E=8, R=2, fp8=True)
