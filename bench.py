@@ -59,22 +59,26 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def source_digest(name):
-    p = os.path.join(HERE, "combine_route_meta_b200", "csrc", name)
-    with open(p, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def source_digest():
+    """Digest of every CUDA source of the library: kernel counters recorded for an
+    older digest no longer describe the kernels."""
+    d = hashlib.sha256()
+    src = os.path.join(HERE, "combine_route_meta_b200", "csrc")
+    for name in sorted(os.listdir(src)):
+        with open(os.path.join(src, name), "rb") as f:
+            d.update(name.encode() + b"\0" + f.read())
+    return d.hexdigest()[:16]
 
 
-def recorded_traffic(kernel_file, workload):
-    """DRAM bytes per launch from a committed ncu summary, if the kernel is unchanged."""
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if the sources are unchanged."""
     p = os.path.join(HERE, "profiles", "dram_traffic.json")
     try:
         with open(p) as f:
             rec = json.load(f)
-        e = rec[kernel_file][workload]
-        if e["source_sha256_16"] != source_digest(kernel_file):
+        if rec["csrc_sha256_16"] != source_digest():
             return None
-        return int(e["bytes_per_launch"])
+        return int(rec["bytes_per_launch"][workload][kernel])
     except Exception:
         return None
 
@@ -207,20 +211,36 @@ def time_oracle(w, budget_s=10.0, max_reps=50):
 
 # ---- GPU arm ----------------------------------------------------------------------------
 
-def count_graph_kernels(g):
-    """Kernel nodes in a captured torch CUDA graph (the launches of one replay)."""
-    from cuda.bindings import runtime as rt
-    graph = rt.cudaGraph_t(init_value=g.raw_cuda_graph())
-    err, _, n = rt.cudaGraphGetNodes(graph, 0)
-    if err != rt.cudaError_t.cudaSuccess:
-        raise RuntimeError(f"cudaGraphGetNodes: {err}")
-    err, nodes, n = rt.cudaGraphGetNodes(graph, n)
-    kernels = 0
+def graph_kernels(g):
+    """Names of the kernel nodes in a captured torch CUDA graph (one replay's launches)."""
+    from cuda.bindings import driver as drv
+    graph = drv.CUgraph(g.raw_cuda_graph())
+    err, _, n = drv.cuGraphGetNodes(graph, 0)
+    if err != drv.CUresult.CUDA_SUCCESS:
+        raise RuntimeError(f"cuGraphGetNodes: {err}")
+    err, nodes, n = drv.cuGraphGetNodes(graph, n)
+    names = []
     for node in nodes[:n]:
-        err, kind = rt.cudaGraphNodeGetType(node)
-        if kind == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel:
-            kernels += 1
-    return kernels
+        err, kind = drv.cuGraphNodeGetType(node)
+        if kind != drv.CUgraphNodeType.CU_GRAPH_NODE_TYPE_KERNEL:
+            continue
+        name = "?"
+        try:
+            err, params = drv.cuGraphKernelNodeGetParams(node)
+            err, raw = drv.cuFuncGetName(params.func)
+            name = raw.decode() if isinstance(raw, bytes) else str(raw)
+        except Exception:
+            pass
+        names.append(name)
+    return names
+
+
+def short_kernel_name(mangled):
+    for k in ("dispatch_fused", "scatter_bulk_bf16", "scatter_rows", "combine_rows",
+              "meta_single_block", "meta_tile_count", "meta_tile_scan", "meta_tile_assign"):
+        if k in mangled:
+            return k
+    return mangled
 
 
 def run_gpu(args, rank, world):
@@ -290,8 +310,16 @@ def run_gpu(args, rank, world):
     g_step = [capture(lambda st=st: (do_dispatch(st), do_combine(st))) for st in sets]
     g_disp = [capture(lambda st=st: do_dispatch(st)) for st in sets]
     g_comb = [capture(lambda st=st: do_combine(st)) for st in sets]
-    launches_per_step = count_graph_kernels(g_step[0])
-    for g in g_step + g_disp + g_comb:
+    step_kernels = [short_kernel_name(k) for k in graph_kernels(g_step[0])]
+    disp_kernels = [short_kernel_name(k) for k in graph_kernels(g_disp[0])]
+    launches_per_step = len(step_kernels)
+    # On the multi-kernel dispatch path the payload kernel is timed on its own too
+    # (moe_dispatch_payload on the slots the last dispatch left).
+    g_pay = None
+    if len(disp_kernels) > 1:
+        g_pay = [capture(lambda st=st: moe.dispatch_payload_into(st.buf, st.x, stream=stream))
+                 for st in sets]
+    for g in g_step + g_disp + g_comb + (g_pay or []):
         g.instantiate()
 
     def run(graphs, n):
@@ -341,6 +369,7 @@ def run_gpu(args, rank, world):
     # Phase split, same protocol: K dispatches alone, then K combines alone.
     disp_ms = run(g_disp, args.steps)
     comb_ms = run(g_comb, args.steps)
+    pay_ms = run(g_pay, args.steps) if g_pay is not None else None
 
     # End to end through the public API with host buffers: H2D of the step's
     # inputs, dispatch, combine, D2H of y, every step.
@@ -373,9 +402,10 @@ def run_gpu(args, rank, world):
         if i >= args.warmup:
             e2e_ms.append(e0.elapsed_time(e1))
 
-    return dict(w=w, total_ms=total_ms, disp_ms=disp_ms, comb_ms=comb_ms, clocks=clocks,
-                launches_per_step=launches_per_step, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h,
-                nsets=nsets, set_bytes=set_bytes, l2=l2)
+    return dict(w=w, total_ms=total_ms, disp_ms=disp_ms, comb_ms=comb_ms, pay_ms=pay_ms,
+                clocks=clocks, launches_per_step=launches_per_step, step_kernels=step_kernels,
+                disp_kernels=disp_kernels, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, nsets=nsets,
+                set_bytes=set_bytes, l2=l2)
 
 
 def main():
@@ -434,14 +464,30 @@ def main():
 
     disp_us = r["disp_ms"] / args.steps * 1e3
     comb_us = r["comb_ms"] / args.steps * 1e3
-    comb_mean_s = comb_us * 1e-6
-    ck_bytes = combine_kernel_bytes(w.T, w.H, w.k)
-    achieved = ck_bytes / comb_mean_s / 1e9
-    roofline = {"bound": "hbm", "kernel": "combine_rows", "achieved": round(achieved, 1),
-                "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                "frac": round(achieved / peak, 4),
-                "traffic": recorded_traffic("combine.cuh", w.name),
-                "algorithmic_bytes": ck_bytes}
+    # Per-kernel rooflines: the dispatch payload kernel (the fused kernel on the
+    # one-launch path) and the combine kernel, each timed alone over K launches.
+    S = w.T * w.k
+    kernels = []
+    if r["pay_ms"] is None:
+        name = r["disp_kernels"][0]
+        kernels.append((name, db, disp_us, "dispatch_fused.cuh"))
+    else:
+        name = ([k for k in r["disp_kernels"] if k.startswith("scatter")] or ["payload"])[-1]
+        pay_bytes = (w.T * w.H * 2 + S * 4
+                     + (S * w.H + S * (w.H // 128) * 4 if w.fp8 else S * w.H * 2))
+        kernels.append((name, pay_bytes, r["pay_ms"] / args.steps * 1e3, "scatter.cuh"))
+    kernels.append(("combine_rows", combine_kernel_bytes(w.T, w.H, w.k), comb_us, "combine.cuh"))
+    per_kernel = []
+    for name, nbytes, us, src in kernels:
+        gbs = nbytes / (us * 1e-6) / 1e9
+        per_kernel.append({"kernel": name, "us": round(us, 3), "algorithmic_bytes": nbytes,
+                           "achieved": round(gbs, 1), "frac": round(gbs / peak, 4),
+                           "traffic": recorded_traffic(name, w.name)})
+    dom = max(per_kernel, key=lambda k: k["us"])
+    roofline = {"bound": "hbm", "kernel": dom["kernel"], "achieved": dom["achieved"],
+                "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": dom["frac"],
+                "traffic": dom["traffic"], "algorithmic_bytes": dom["algorithmic_bytes"],
+                "kernels": per_kernel}
     e2e_s = statistics.median(r["e2e_ms"]) * 1e-3
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
@@ -465,6 +511,7 @@ def main():
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                 "ms_per_step": round(e2e_s * 1e3, 4)},
         "gpu_launches": r["launches_per_step"] * args.steps,
+        "kernels_per_step": r["step_kernels"],
         "clocks": r["clocks"],
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -89,6 +89,11 @@ def _declare(lib):
     lib.moe_dispatch.argtypes = [cfgp, i32, P, P, P, ctypes.POINTER(moe_dispatch_out), P, P,
                                  ctypes.c_size_t, P, P, ctypes.POINTER(moe_handle)]
     lib.moe_dispatch.restype = ctypes.c_int
+    lib.moe_dispatch_layout.argtypes = [cfgp, i32, P, ctypes.POINTER(moe_dispatch_out), P, P,
+                                        ctypes.c_size_t, P, P]
+    lib.moe_dispatch_layout.restype = ctypes.c_int
+    lib.moe_dispatch_payload.argtypes = [cfgp, i32, P, P, ctypes.POINTER(moe_dispatch_out), P, P]
+    lib.moe_dispatch_payload.restype = ctypes.c_int
     lib.moe_dispatch_no_alloc.argtypes = [cfgp, i32, P, P, P, ctypes.POINTER(moe_dispatch_out), P,
                                           P, P, ctypes.POINTER(moe_handle)]
     lib.moe_dispatch_no_alloc.restype = ctypes.c_int
@@ -111,6 +116,8 @@ moe_workspace_bytes = lib.moe_workspace_bytes
 moe_dispatch_sizes_for = lib.moe_dispatch_sizes_for
 moe_dispatch = lib.moe_dispatch
 moe_dispatch_no_alloc = lib.moe_dispatch_no_alloc
+moe_dispatch_layout = lib.moe_dispatch_layout
+moe_dispatch_payload = lib.moe_dispatch_payload
 moe_combine = lib.moe_combine
 moe_check = lib.moe_check
 moe_selftest_bounded_wait = lib.moe_selftest_bounded_wait
@@ -244,6 +251,28 @@ def dispatch_into(buf: Buffers, x: torch.Tensor, topk_idx: torch.Tensor, topk_w:
                           ctypes.c_void_p(buf.err.data_ptr()), ctypes.c_void_p(_stream_ptr(stream)),
                           ctypes.byref(buf.handle_c))
     _ok(st, "moe_dispatch")
+
+
+def dispatch_layout_into(buf: Buffers, topk_idx: torch.Tensor,
+                         stream: Optional[torch.cuda.Stream] = None) -> None:
+    """moe_dispatch_layout: counts, offsets, slots and recv_src only."""
+    st = lib.moe_dispatch_layout(ctypes.byref(buf.cfg), buf.T, ctypes.c_void_p(topk_idx.data_ptr()),
+                                 ctypes.byref(buf.out), ctypes.c_void_p(buf.slot.data_ptr()),
+                                 ctypes.c_void_p(buf.workspace.data_ptr()), buf.workspace_bytes,
+                                 ctypes.c_void_p(buf.err.data_ptr()),
+                                 ctypes.c_void_p(_stream_ptr(stream)))
+    _ok(st, "moe_dispatch_layout")
+
+
+def dispatch_payload_into(buf: Buffers, x: torch.Tensor, slot: Optional[torch.Tensor] = None,
+                          stream: Optional[torch.cuda.Stream] = None) -> None:
+    """moe_dispatch_payload: the rows of x to the slots (buf.slot by default)."""
+    slot = buf.slot if slot is None else slot
+    st = lib.moe_dispatch_payload(ctypes.byref(buf.cfg), buf.T, ctypes.c_void_p(x.data_ptr()),
+                                  ctypes.c_void_p(slot.data_ptr()), ctypes.byref(buf.out),
+                                  ctypes.c_void_p(buf.err.data_ptr()),
+                                  ctypes.c_void_p(_stream_ptr(stream)))
+    _ok(st, "moe_dispatch_payload")
 
 
 def combine_into(handle_c: moe_handle, expert_out: torch.Tensor, y: torch.Tensor,

@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_fused(FusedArgs 
     for (int i = 0; i < kChunks; ++i) {
         const int32_t c = warp + i * nwarps;
         if (c < chunks)
-            store_chunk<L, kFp8>(a.recv_x, a.recv_scale, a.H, c, a.k, s_slot, d[i]);
+            store_chunk<L, kFp8>(a.recv_x, a.recv_scale, a.H, c, a.k, s_slot, a.rows_cap, a.err, d[i]);
     }
 }
 

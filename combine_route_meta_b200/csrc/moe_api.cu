@@ -196,6 +196,117 @@ unsigned grid_for(int64_t units, int sms, int ctas_per_sm)
     return (unsigned)(g > 0 ? g : 1);
 }
 
+// Argument checks of the layout phase (shared by moe_dispatch).
+int check_layout_args(const moe_config *cfg, int32_t T, const int32_t *topk_idx,
+                      const moe_dispatch_out *out, const int32_t *slot, const void *workspace,
+                      size_t workspace_bytes_given, const int32_t *dev_err)
+{
+    if (T < 0 || out == nullptr || dev_err == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    const int64_t S = (int64_t)T * cfg->k;
+    const int64_t rows_cap = out->rows_cap;
+    if (rows_cap < 0 || rows_cap > INT32_MAX || S > INT32_MAX)
+        return MOE_ERR_INVALID_ARG;
+    if (rows_capacity(cfg, T) > INT32_MAX)
+        return MOE_ERR_UNSUPPORTED;
+    if (out->expert_count == nullptr || out->expert_offset == nullptr ||
+        out->rank_offset == nullptr || (rows_cap > 0 && out->recv_src == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (topk_idx == nullptr || slot == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    const size_t need_ws = workspace_bytes(cfg, T);
+    if (need_ws > 0 && (workspace == nullptr || workspace_bytes_given < need_ws))
+        return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+// Argument checks of the payload phase (shared by moe_dispatch).
+int check_payload_args(const moe_config *cfg, int32_t T, const void *x, const int32_t *slot,
+                       const moe_dispatch_out *out)
+{
+    const bool fp8 = cfg->flags & MOE_FP8;
+    if (T < 0 || out == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (x == nullptr || slot == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    if (out->rows_cap > 0 && (out->recv_x == nullptr || (fp8 && out->recv_scale == nullptr)))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(out->recv_x) || (fp8 && !aligned16(out->recv_scale)))
+        return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+// Routing metadata without payload: one CTA for small batches, tiled otherwise.
+int launch_layout(const moe_config *cfg, int32_t T, const int32_t *topk_idx,
+                  const moe_dispatch_out *out, int32_t *slot, void *workspace, int32_t *dev_err,
+                  cudaStream_t s)
+{
+    MetaArgs m;
+    m.topk_idx = topk_idx;
+    m.S = (int64_t)T * cfg->k;
+    m.k = cfg->k;
+    m.E = cfg->E;
+    m.R = cfg->R;
+    m.pad128 = (cfg->flags & MOE_PAD128) ? 1 : 0;
+    m.rows_cap = out->rows_cap;
+    m.expert_count = out->expert_count;
+    m.expert_offset = out->expert_offset;
+    m.rank_offset = out->rank_offset;
+    m.slot = slot;
+    m.recv_src = out->recv_src;
+    m.err = dev_err;
+    if (use_single_block(m.S))
+        return launched(launch(meta_single_block, 1, kMetaThreads, meta_single_smem(cfg->E), s, m));
+    const int64_t ntiles = meta_tiles(m.S);
+    int32_t *tile_hist = static_cast<int32_t *>(workspace);
+    const int32_t *tile_prefix = tile_hist;
+    int st;
+    if ((st = launched(launch(meta_tile_count, (unsigned)ntiles, kMetaThreads, meta_count_smem(cfg->E),
+                              s, m, tile_hist))) != MOE_OK ||
+        (st = launched(launch(meta_tile_scan, (unsigned)((cfg->E + kWarp - 1) / kWarp), kScanThreads,
+                              0, s, m, tile_hist, (int32_t)ntiles))) != MOE_OK ||
+        (st = launched(launch(meta_tile_assign, (unsigned)ntiles, kMetaThreads,
+                              meta_assign_smem(cfg->E), s, m, tile_prefix))) != MOE_OK)
+        return st;
+    return MOE_OK;
+}
+
+// Payload rows to the slots: bulk copies for bf16 rows of at least 1 KB,
+// register stores (and the fp8 quantiser) otherwise.
+int launch_payload(const moe_config *cfg, int32_t T, const void *x, const int32_t *slot,
+                   const moe_dispatch_out *out, int32_t *dev_err, const DeviceInfo *dev,
+                   cudaStream_t s)
+{
+    if (T == 0)
+        return MOE_OK;
+    const bool fp8 = cfg->flags & MOE_FP8;
+    ScatterArgs a;
+    a.x = static_cast<const uint16_t *>(x);
+    a.slot = slot;
+    a.T = T;
+    a.H = cfg->H;
+    a.k = cfg->k;
+    a.rows_cap = out->rows_cap;
+    a.recv_x = out->recv_x;
+    a.recv_scale = out->recv_scale;
+    a.err = dev_err;
+    cudaError_t e;
+    if (use_bulk_scatter(cfg->H, fp8)) {
+        const unsigned grid = grid_for(T, dev->sms, kBulkCtasPerSm);
+        const size_t smem = (size_t)kBulkStages * bulk_stage_bytes(cfg->H);
+        e = launch(scatter_bulk_bf16, grid, kWarp, smem, s, a);
+    } else {
+        constexpr int kCols = chunk_cols<kScatterLaneCols>();
+        const int64_t warp_units = (int64_t)T * ((cfg->H + kCols - 1) / kCols);
+        const int warps_per_cta = kScatterThreads / kWarp;
+        const unsigned grid = grid_for((warp_units + warps_per_cta - 1) / warps_per_cta, dev->sms,
+                                       2048 / kScatterThreads);
+        e = fp8 ? launch(scatter_rows<true>, grid, kScatterThreads, 0, s, a)
+                : launch(scatter_rows<false>, grid, kScatterThreads, 0, s, a);
+    }
+    return launched(e);
+}
+
 } // namespace
 } // namespace moe
 
@@ -266,47 +377,17 @@ int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
     int st = check_config(cfg);
     if (st != MOE_OK)
         return st;
-    if (T < 0 || out == nullptr || handle == nullptr || dev_err == nullptr)
+    if (handle == nullptr || (T > 0 && topk_w == nullptr))
         return MOE_ERR_INVALID_ARG;
-    const bool fp8 = cfg->flags & MOE_FP8;
-    const int64_t S = (int64_t)T * cfg->k;
-    const int64_t rows_cap = out->rows_cap;
-    if (rows_cap < 0 || rows_cap > INT32_MAX || S > INT32_MAX)
-        return MOE_ERR_INVALID_ARG;
-    if (rows_capacity(cfg, T) > INT32_MAX)
-        return MOE_ERR_UNSUPPORTED;
-    if (out->expert_count == nullptr || out->expert_offset == nullptr ||
-        out->rank_offset == nullptr || (rows_cap > 0 && out->recv_src == nullptr))
-        return MOE_ERR_INVALID_ARG;
-    if (T > 0 && (x == nullptr || topk_idx == nullptr || topk_w == nullptr || slot == nullptr))
-        return MOE_ERR_INVALID_ARG;
-    if (rows_cap > 0 && (out->recv_x == nullptr || (fp8 && out->recv_scale == nullptr)))
-        return MOE_ERR_INVALID_ARG;
-    if (!aligned16(x) || !aligned16(out->recv_x) || (fp8 && !aligned16(out->recv_scale)))
-        return MOE_ERR_INVALID_ARG;
-    const size_t need_ws = workspace_bytes(cfg, T);
-    if (need_ws > 0 && (workspace == nullptr || workspace_bytes_given < need_ws))
-        return MOE_ERR_INVALID_ARG;
-
+    if ((st = check_layout_args(cfg, T, topk_idx, out, slot, workspace, workspace_bytes_given,
+                                dev_err)) != MOE_OK ||
+        (st = check_payload_args(cfg, T, x, slot, out)) != MOE_OK)
+        return st;
     DeviceInfo *dev = nullptr;
     if ((st = device_info(&dev)) != MOE_OK)
         return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-
-    MetaArgs m;
-    m.topk_idx = topk_idx;
-    m.S = S;
-    m.k = cfg->k;
-    m.E = cfg->E;
-    m.R = cfg->R;
-    m.pad128 = (cfg->flags & MOE_PAD128) ? 1 : 0;
-    m.rows_cap = rows_cap;
-    m.expert_count = out->expert_count;
-    m.expert_offset = out->expert_offset;
-    m.rank_offset = out->rank_offset;
-    m.slot = slot;
-    m.recv_src = out->recv_src;
-    m.err = dev_err;
+    const bool fp8 = cfg->flags & MOE_FP8;
 
     unsigned fused_block = 0;
     if (const int per = fused_chunks(cfg, T, &fused_block)) {
@@ -318,8 +399,8 @@ int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
         f.k = cfg->k;
         f.E = cfg->E;
         f.R = cfg->R;
-        f.pad128 = m.pad128;
-        f.rows_cap = rows_cap;
+        f.pad128 = (cfg->flags & MOE_PAD128) ? 1 : 0;
+        f.rows_cap = out->rows_cap;
         f.recv_x = out->recv_x;
         f.recv_scale = out->recv_scale;
         f.expert_count = out->expert_count;
@@ -333,64 +414,50 @@ int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
                 : launch_fused<false>(per, T, fused_block, fused_smem(cfg->E), s, f);
         if ((st = launched(e)) != MOE_OK)
             return st;
-        handle->cfg = *cfg;
-        handle->T = T;
-        handle->slot = slot;
-        handle->topk_w = topk_w;
-        handle->rows_cap = rows_cap;
-        return MOE_OK;
-    }
-
-    if (use_single_block(S)) {
-        if ((st = launched(launch(meta_single_block, 1, kMetaThreads, meta_single_smem(cfg->E), s,
-                                  m))) != MOE_OK)
-            return st;
     } else {
-        const int64_t ntiles = meta_tiles(S);
-        int32_t *tile_hist = static_cast<int32_t *>(workspace);
-        const int32_t *tile_prefix = tile_hist;
-        if ((st = launched(launch(meta_tile_count, (unsigned)ntiles, kMetaThreads,
-                                  meta_count_smem(cfg->E), s, m, tile_hist))) != MOE_OK ||
-            (st = launched(launch(meta_tile_scan, (unsigned)((cfg->E + kWarp - 1) / kWarp),
-                                  kScanThreads, 0, s, m, tile_hist, (int32_t)ntiles))) != MOE_OK ||
-            (st = launched(launch(meta_tile_assign, (unsigned)ntiles, kMetaThreads,
-                                  meta_assign_smem(cfg->E), s, m, tile_prefix))) != MOE_OK)
+        if ((st = launch_layout(cfg, T, topk_idx, out, slot, workspace, dev_err, s)) != MOE_OK ||
+            (st = launch_payload(cfg, T, x, slot, out, dev_err, dev, s)) != MOE_OK)
             return st;
     }
-
-    if (T > 0) {
-        ScatterArgs a;
-        a.x = static_cast<const uint16_t *>(x);
-        a.slot = slot;
-        a.T = T;
-        a.H = cfg->H;
-        a.k = cfg->k;
-        a.recv_x = out->recv_x;
-        a.recv_scale = out->recv_scale;
-        cudaError_t e;
-        if (use_bulk_scatter(cfg->H, fp8)) {
-            const unsigned grid = grid_for(T, dev->sms, kBulkCtasPerSm);
-            const size_t smem = (size_t)kBulkStages * bulk_stage_bytes(cfg->H);
-            e = launch(scatter_bulk_bf16, grid, kWarp, smem, s, a, dev_err);
-        } else {
-            constexpr int kCols = chunk_cols<kScatterLaneCols>();
-            const int64_t warp_units = (int64_t)T * ((cfg->H + kCols - 1) / kCols);
-            const int warps_per_cta = kScatterThreads / kWarp;
-            const unsigned grid = grid_for((warp_units + warps_per_cta - 1) / warps_per_cta, dev->sms,
-                                           2048 / kScatterThreads);
-            e = fp8 ? launch(scatter_rows<true>, grid, kScatterThreads, 0, s, a)
-                    : launch(scatter_rows<false>, grid, kScatterThreads, 0, s, a);
-        }
-        if ((st = launched(e)) != MOE_OK)
-            return st;
-    }
-
     handle->cfg = *cfg;
     handle->T = T;
     handle->slot = slot;
     handle->topk_w = topk_w;
-    handle->rows_cap = rows_cap;
+    handle->rows_cap = out->rows_cap;
     return MOE_OK;
+}
+
+int moe_dispatch_layout(const moe_config *cfg, int32_t T, const int32_t *topk_idx,
+                        const moe_dispatch_out *out, int32_t *slot, void *workspace,
+                        size_t workspace_bytes_given, int32_t *dev_err, void *stream)
+{
+    int st = check_config(cfg);
+    if (st != MOE_OK)
+        return st;
+    if ((st = check_layout_args(cfg, T, topk_idx, out, slot, workspace, workspace_bytes_given,
+                                dev_err)) != MOE_OK)
+        return st;
+    DeviceInfo *dev = nullptr;
+    if ((st = device_info(&dev)) != MOE_OK)
+        return st;
+    return launch_layout(cfg, T, topk_idx, out, slot, workspace, dev_err,
+                         static_cast<cudaStream_t>(stream));
+}
+
+int moe_dispatch_payload(const moe_config *cfg, int32_t T, const void *x, const int32_t *slot,
+                         const moe_dispatch_out *out, int32_t *dev_err, void *stream)
+{
+    int st = check_config(cfg);
+    if (st != MOE_OK)
+        return st;
+    if (dev_err == nullptr || out == nullptr || out->rows_cap < 0 || out->rows_cap > INT32_MAX)
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_payload_args(cfg, T, x, slot, out)) != MOE_OK)
+        return st;
+    DeviceInfo *dev = nullptr;
+    if ((st = device_info(&dev)) != MOE_OK)
+        return st;
+    return launch_payload(cfg, T, x, slot, out, dev_err, dev, static_cast<cudaStream_t>(stream));
 }
 
 int moe_combine(const moe_handle *handle, const void *expert_out, void *y, int32_t *dev_err,

@@ -37,12 +37,26 @@ template <int kLaneCols>
 __host__ __device__ constexpr int chunk_cols() { return 32 * kLaneCols; }
 
 struct ScatterArgs {
-    const uint16_t *x; // [T, H] bf16
-    const int32_t *slot; // [T, k]
+    const uint16_t *x;   // [T, H] bf16
+    const int32_t *slot; // [T, k]: receive row of each entry, -1 = none
     int32_t T, H, k;
-    void *recv_x; // [rows_cap, H] bf16 or e4m3
-    float *recv_scale; // [rows_cap, H/128] (fp8)
+    int64_t rows_cap;    // slots at or past it are skipped and flagged
+    void *recv_x;        // [rows_cap, H] bf16 or e4m3
+    float *recv_scale;   // [rows_cap, H/128] (fp8)
+    int32_t *err;
 };
+
+// The receive row of slot value s, or -1 for "no row"; a value outside
+// [-1, rows_cap) is flagged and skipped, so a bad slot array never writes out
+// of bounds.
+__device__ __forceinline__ int32_t checked_slot(int32_t s, int64_t rows_cap, int32_t *err)
+{
+    if (s >= 0 && s < rows_cap)
+        return s;
+    if (s != -1)
+        raise_error(err, MOE_DEV_BAD_SLOT);
+    return -1;
+}
 
 // The lane's columns of one chunk: kLaneCols/8 vectors of 8 bf16.
 template <int kLaneCols>
@@ -148,8 +162,8 @@ __device__ __forceinline__ void load_chunk(const uint16_t *xr, int32_t H, int32_
 // or shared memory.
 template <int kLaneCols, bool kFp8>
 __device__ __forceinline__ void store_chunk(void *recv_x, float *recv_scale, int32_t H, int32_t c,
-                                            int32_t k, const int32_t *slots,
-                                            const LaneData<kLaneCols> &d)
+                                            int32_t k, const int32_t *slots, int64_t rows_cap,
+                                            int32_t *err, const LaneData<kLaneCols> &d)
 {
     const unsigned lane = lane_id();
     if constexpr (kFp8) {
@@ -168,7 +182,8 @@ __device__ __forceinline__ void store_chunk(void *recv_x, float *recv_scale, int
         const bool scale_vec = (nb % kBlocks == 0) && (c * kBlocks + kBlocks - 1 < nb);
         uint8_t *rx = static_cast<uint8_t *>(recv_x);
         for (int32_t j0 = 0; j0 < k; j0 += kWarp) {
-            const int32_t my = j0 + (int32_t)lane < k ? slots[j0 + lane] : -1;
+            const int32_t my =
+                j0 + (int32_t)lane < k ? checked_slot(slots[j0 + lane], rows_cap, err) : -1;
             const int32_t jn = k - j0 < kWarp ? k - j0 : kWarp;
             for (int32_t j = 0; j < jn; ++j) {
                 const int32_t s = __shfl_sync(kFullMask, my, j);
@@ -198,7 +213,8 @@ __device__ __forceinline__ void store_chunk(void *recv_x, float *recv_scale, int
     } else {
         uint16_t *rx = static_cast<uint16_t *>(recv_x);
         for (int32_t j0 = 0; j0 < k; j0 += kWarp) {
-            const int32_t my = j0 + (int32_t)lane < k ? slots[j0 + lane] : -1;
+            const int32_t my =
+                j0 + (int32_t)lane < k ? checked_slot(slots[j0 + lane], rows_cap, err) : -1;
             const int32_t jn = k - j0 < kWarp ? k - j0 : kWarp;
             for (int32_t j = 0; j < jn; ++j) {
                 const int32_t s = __shfl_sync(kFullMask, my, j);
@@ -230,7 +246,8 @@ __global__ void __launch_bounds__(kScatterThreads) scatter_rows(ScatterArgs a)
         const int32_t c = (int32_t)(u % chunks);
         LaneData<L> d;
         load_chunk<L, kFp8>(a.x + (int64_t)t * a.H, a.H, c, d);
-        store_chunk<L, kFp8>(a.recv_x, a.recv_scale, a.H, c, a.k, a.slot + (int64_t)t * a.k, d);
+        store_chunk<L, kFp8>(a.recv_x, a.recv_scale, a.H, c, a.k, a.slot + (int64_t)t * a.k,
+                             a.rows_cap, a.err, d);
     }
 }
 
@@ -257,7 +274,7 @@ __host__ __device__ inline uint32_t bulk_stage_bytes(int32_t H)
     return ((uint32_t)H * 2 + 127) / 128 * 128;
 }
 
-__global__ void __launch_bounds__(kWarp) scatter_bulk_bf16(ScatterArgs a, int32_t *err)
+__global__ void __launch_bounds__(kWarp) scatter_bulk_bf16(ScatterArgs a)
 {
     stream_order_begin();
     extern __shared__ __align__(128) uint8_t stage_mem[];
@@ -289,12 +306,12 @@ __global__ void __launch_bounds__(kWarp) scatter_bulk_bf16(ScatterArgs a, int32_
         const int s = (int)(i % kBulkStages);
         if (!mbar_wait(smem_addr(&bars[s]), (uint32_t)((i / kBulkStages) & 1), kWaitLimitNs)) {
             if (lane == 0)
-                raise_error(err, MOE_DEV_TIMEOUT);
+                raise_error(a.err, MOE_DEV_TIMEOUT);
             break;
         }
         const int32_t t = token(i);
         for (int32_t j = (int32_t)lane; j < a.k; j += kWarp) {
-            const int32_t d = __ldg(a.slot + (int64_t)t * a.k + j);
+            const int32_t d = checked_slot(__ldg(a.slot + (int64_t)t * a.k + j), a.rows_cap, a.err);
             if (d >= 0)
                 bulk_store(static_cast<uint16_t *>(a.recv_x) + (int64_t)d * a.H,
                            smem_addr(stage_mem + s * stage_bytes), row);

@@ -71,7 +71,7 @@ extern "C" {
 #define MOE_DEV_BAD_INDEX 1 /* dispatch: an expert id outside [0, E)                  */
 #define MOE_DEV_CAPACITY 2  /* dispatch: a receive row at or past rows_cap            */
 #define MOE_DEV_TIMEOUT 4   /* a bounded device wait (1 s) gave up                     */
-#define MOE_DEV_BAD_SLOT 8  /* combine: a slot outside [-1, rows_cap) in the handle   */
+#define MOE_DEV_BAD_SLOT 8  /* payload / combine: a slot outside [-1, rows_cap)        */
 
 /* Limits of this build. */
 #define MOE_MAX_EXPERTS 2048 /* E */
@@ -182,6 +182,32 @@ MOE_API int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const 
                  const float *topk_w, const moe_dispatch_out *out, int32_t *slot,
                  void *workspace, size_t workspace_bytes, int32_t *dev_err, void *stream,
                  moe_handle *handle);
+
+/*
+ * The two phases of moe_dispatch as separate calls, in the order of the EFA
+ * page's section "Despacho e Combinação" (routing information first: counts,
+ * their cumulative sum and the offsets that place each token; then the
+ * payload is packed).  moe_dispatch_layout followed by moe_dispatch_payload
+ * gives exactly the results of moe_dispatch.
+ *
+ * moe_dispatch_layout: the per-expert counts, offsets, rank offsets, slot[T,k]
+ * and recv_src of moe_dispatch; it reads only topk_idx and writes only those
+ * arrays of `out` (recv_x / recv_scale may be NULL).  Same workspace rules.
+ *
+ * moe_dispatch_payload: copies (bf16) or block-quantises (MOE_FP8) each token's
+ * row x[t] into rows slot[t, 0..k) of out->recv_x (and out->recv_scale).  The
+ * slots normally come from a layout call with the same cfg, T and
+ * out->rows_cap.  A slot of -1 is skipped; any other value outside
+ * [0, rows_cap) is skipped and sets MOE_DEV_BAD_SLOT, so no write leaves the
+ * buffers.  It uses only recv_x, recv_scale and rows_cap of `out`.
+ */
+MOE_API int moe_dispatch_layout(const moe_config *cfg, int32_t T, const int32_t *topk_idx,
+                                const moe_dispatch_out *out, int32_t *slot, void *workspace,
+                                size_t workspace_bytes, int32_t *dev_err, void *stream);
+
+MOE_API int moe_dispatch_payload(const moe_config *cfg, int32_t T, const void *x,
+                                 const int32_t *slot, const moe_dispatch_out *out,
+                                 int32_t *dev_err, void *stream);
 
 /*
  * Combine (EFA page, sections "Introdução" and "Despacho e Combinação"; DeepSeek

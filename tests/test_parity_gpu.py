@@ -383,3 +383,50 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     # the context is still usable: a normal dispatch + combine matches the oracle
     x, idx, w = random_problem(12, 64, 512, 8, 2)
     check_problem(x, idx, w, E=8, R=2, fp8=True)
+
+
+@pytest.mark.parametrize("T,H,E,k,fp8,pad128", [(40, 256, 8, 4, True, False),       # one-CTA layout
+                                                (3000, 1024, 64, 8, False, True),   # tiled, bulk bf16
+                                                (700, 7168, 256, 8, True, True)])   # tiled, fp8
+def test_layout_then_payload_equals_dispatch(T, H, E, k, fp8, pad128):
+    x, idx, w = random_problem(T + H, T, H, E, k)
+    ref, bits, _ = run_gpu(x, idx, w, E=E, R=E // 4 or 1, fp8=fp8, pad128=pad128)
+    assert bits == 0
+    cfg = moe.make_config(H, k, E, E // 4 or 1, fp8, pad128)
+    buf = moe.Buffers(cfg, T, "cuda")
+    buf.recv_x.view(torch.uint8).fill_(POISON)
+    if buf.recv_scale is not None:
+        buf.recv_scale.view(torch.uint8).fill_(POISON)
+    idd, xd = to_dev(idx), bf16_to_dev(x)
+    moe.dispatch_layout_into(buf, idd)
+    moe.dispatch_payload_into(buf, xd)
+    assert moe.check() == 0
+    a, b = dispatch_host(buf), dispatch_host(ref)
+    for key in a:
+        np.testing.assert_array_equal(a[key], b[key], err_msg=key)
+
+
+@pytest.mark.parametrize("H,fp8", [(256, False), (2048, False), (512, True)])
+def test_payload_skips_and_flags_bad_slots(H, fp8):
+    # register scatter (H=256), bulk scatter (bf16, H=2048) and fp8: slots outside
+    # [-1, rows_cap) are skipped and flagged; nothing outside the buffers is touched
+    T, k = 20, 2
+    x, _, _ = random_problem(3, T, H, 8, k)
+    cfg = moe.make_config(H, k, 8, 2, fp8)
+    buf = moe.Buffers(cfg, T, "cuda", rows_cap=T * k)
+    buf.recv_x.view(torch.uint8).fill_(POISON)
+    slot = np.arange(T * k, dtype=np.int32).reshape(T, k)
+    slot[3, 1] = T * k          # one past the end
+    slot[5, 0] = -7             # negative, not -1
+    slot[6, 1] = -1             # "no row": skipped silently
+    moe.check()
+    moe.dispatch_payload_into(buf, bf16_to_dev(x), to_dev(slot))
+    assert moe.check() == moe.DEV_BAD_SLOT
+    got = buf.recv_x.view(torch.uint8).cpu().numpy().reshape(T * k, -1)
+    # each row r was meant for entry r; the three entries without a valid slot left theirs alone
+    for r in (3 * k + 1, 5 * k + 0, 6 * k + 1):
+        assert np.all(got[r] == POISON), r
+    if not fp8:
+        for t in (0, 7, T - 1):
+            for j in range(k):
+                np.testing.assert_array_equal(got[slot[t, j]].view(np.uint16), x[t])
