@@ -211,6 +211,19 @@ def time_oracle(w, budget_s=10.0, max_reps=50):
 
 # ---- GPU arm ----------------------------------------------------------------------------
 
+def max_over_ranks(value, dist, device):
+    """The largest of every rank's value (all ranks take part and all get it)."""
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(step_bytes, world, ms_per_step):
+    """Whole-job GB/s: every rank moves step_bytes per step (weak scaling)."""
+    return step_bytes * world / (ms_per_step * 1e-3) / 1e9
+
+
 def graph_kernels(g):
     """Names of the kernel nodes in a captured torch CUDA graph (one replay's launches)."""
     from cuda.bindings import driver as drv
@@ -362,9 +375,7 @@ def run_gpu(args, rank, world):
     if bits:
         raise RuntimeError(f"device error bits {bits} during timing")
     if dist is not None:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+        total_ms = max_over_ranks(total_ms, dist, dev)
 
     # Phase split, same protocol: K dispatches alone, then K combines alone.
     disp_ms = run(g_disp, args.steps)
@@ -460,7 +471,7 @@ def main():
     db, cb = algorithmic_bytes(w.T, w.H, w.E, w.R, w.k, w.fp8)
     step_bytes = db + cb
     ms_per_step = r["total_ms"] / args.steps
-    value = step_bytes * world / (ms_per_step * 1e-3) / 1e9
+    value = job_throughput(step_bytes, world, ms_per_step)
 
     disp_us = r["disp_ms"] / args.steps * 1e3
     comb_us = r["comb_ms"] / args.steps * 1e3
