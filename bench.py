@@ -313,37 +313,62 @@ def run_gpu(args, rank, world):
     if moe.check(stream) != 0:
         raise RuntimeError("device error during warm-up")
 
-    # One CUDA graph per set and phase (the step graph holds dispatch + combine).
-    def capture(fn):
+    # CUDA graphs.  A top-level submission (a kernel launch or a graph launch)
+    # costs about 2 us on this GPU however small its work, while a kernel
+    # boundary inside a graph costs well under 1 us; a serving engine captures a
+    # whole forward pass.  So one graph holds a rotation of steps, one per input
+    # set (a step = dispatch + combine on that set), and K steps are replayed as
+    # whole rotations plus one graph with the remainder.
+    def capture(fns):
         g = torch.cuda.CUDAGraph(keep_graph=True)
         with torch.cuda.graph(g, stream=stream):
-            fn()
+            for fn in fns:
+                fn()
         return g
 
-    g_step = [capture(lambda st=st: (do_dispatch(st), do_combine(st))) for st in sets]
-    g_disp = [capture(lambda st=st: do_dispatch(st)) for st in sets]
-    g_comb = [capture(lambda st=st: do_combine(st)) for st in sets]
-    step_kernels = [short_kernel_name(k) for k in graph_kernels(g_step[0])]
-    disp_kernels = [short_kernel_name(k) for k in graph_kernels(g_disp[0])]
-    launches_per_step = len(step_kernels)
-    # On the multi-kernel dispatch path the payload kernel is timed on its own too
-    # (moe_dispatch_payload on the slots the last dispatch left).
-    g_pay = None
-    if len(disp_kernels) > 1:
-        g_pay = [capture(lambda st=st: moe.dispatch_payload_into(st.buf, st.x, stream=stream))
-                 for st in sets]
-    for g in g_step + g_disp + g_comb + (g_pay or []):
-        g.instantiate()
+    def rotation(make, count):
+        return capture([make(sets[i % nsets]) for i in range(count)])
 
-    def run(graphs, n):
-        """Replays n graphs back to back (rotating sets); device milliseconds."""
+    step_fn = lambda st: (lambda: (do_dispatch(st), do_combine(st)))
+    disp_fn = lambda st: (lambda: do_dispatch(st))
+    comb_fn = lambda st: (lambda: do_combine(st))
+    pay_fn = lambda st: (lambda: moe.dispatch_payload_into(st.buf, st.x, stream=stream))
+
+    g_one = rotation(step_fn, 1)
+    step_kernels = [short_kernel_name(k) for k in graph_kernels(g_one)]
+    disp_kernels = [short_kernel_name(k) for k in graph_kernels(rotation(disp_fn, 1))]
+    launches_per_step = len(step_kernels)
+    graph_cache = {}
+
+    per_graph = max(nsets, 8)
+
+    def graphs_for(name, make, n):
+        """(full-rotation graph, remainder graph or None, rotations) covering n steps."""
+        q, r = divmod(n, per_graph)
+        key = (name, r)
+        if key not in graph_cache:
+            full = rotation(make, per_graph)
+            full.instantiate()
+            rest = None
+            if r:
+                rest = rotation(make, r)
+                rest.instantiate()
+            graph_cache[key] = (full, rest)
+        full, rest = graph_cache[key]
+        return full, rest, q
+
+    def run(name, make, n):
+        """Runs n steps of `make` back to back (rotating sets); device milliseconds."""
+        full, rest, q = graphs_for(name, make, n)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
             # a sleeping kernel in front lets the host queue the replays ahead of the GPU
-            torch.cuda._sleep(min(n, 256) * 20_000)
+            torch.cuda._sleep(min(q + 1, 256) * 100_000)
             e0.record(stream)
-            for i in range(n):
-                graphs[i % nsets].replay()
+            for _ in range(q):
+                full.replay()
+            if rest is not None:
+                rest.replay()
             e1.record(stream)
         e1.synchronize()
         return e0.elapsed_time(e1)
@@ -353,9 +378,10 @@ def run_gpu(args, rank, world):
     sampler = ClockSampler(dev.index)
     sampler.start()
     t_warm = time.monotonic()
-    run(g_step, max(args.warmup, nsets))
+    run("step", step_fn, max(args.warmup, per_graph))
     while sampler.count() < 3 and time.monotonic() - t_warm < 5.0:
-        run(g_step, 200)
+        run("step", step_fn, 20 * per_graph)
+    graphs_for("step", step_fn, args.steps)  # capture before the timed region
     torch.cuda.synchronize()
 
     dist = None
@@ -364,7 +390,7 @@ def run_gpu(args, rank, world):
         dist.barrier()
     torch.cuda.synchronize()
     sampler.mark_start()
-    total_ms = run(g_step, args.steps)
+    total_ms = run("step", step_fn, args.steps)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
@@ -377,10 +403,12 @@ def run_gpu(args, rank, world):
     if dist is not None:
         total_ms = max_over_ranks(total_ms, dist, dev)
 
-    # Phase split, same protocol: K dispatches alone, then K combines alone.
-    disp_ms = run(g_disp, args.steps)
-    comb_ms = run(g_comb, args.steps)
-    pay_ms = run(g_pay, args.steps) if g_pay is not None else None
+    # Phase split, same protocol: K dispatches alone, K combines alone, and on the
+    # multi-kernel dispatch path K payload kernels alone (moe_dispatch_payload on
+    # the slots the last dispatch of each set left).
+    disp_ms = run("disp", disp_fn, args.steps)
+    comb_ms = run("comb", comb_fn, args.steps)
+    pay_ms = run("pay", pay_fn, args.steps) if len(disp_kernels) > 1 else None
 
     # End to end through the public API with host buffers: H2D of the step's
     # inputs, dispatch, combine, D2H of y, every step.
@@ -416,7 +444,7 @@ def run_gpu(args, rank, world):
     return dict(w=w, total_ms=total_ms, disp_ms=disp_ms, comb_ms=comb_ms, pay_ms=pay_ms,
                 clocks=clocks, launches_per_step=launches_per_step, step_kernels=step_kernels,
                 disp_kernels=disp_kernels, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, nsets=nsets,
-                set_bytes=set_bytes, l2=l2)
+                set_bytes=set_bytes, l2=l2, per_graph=per_graph)
 
 
 def main():
@@ -511,7 +539,8 @@ def main():
                    "l2": (f"{r['nsets']} rotating sets of {r['set_bytes'] / 1e6:.1f} MB "
                           f"({r['nsets'] * r['set_bytes'] / 1e6:.0f} MB touched between uses of a "
                           f"set; L2 {r['l2'] / 1e6:.0f} MB)"),
-                   "graphs": "one CUDA graph per step, replayed back to back",
+                   "graphs": (f"CUDA graphs of {r['per_graph']} steps over the rotating sets, "
+                              "replayed back to back"),
                    "parallelism": f"replicas x{world}"},
         "dispatch_us": round(disp_us, 2), "combine_us": round(comb_us, 2),
         "total_us": round(ms_per_step * 1e3, 2),

@@ -11,7 +11,7 @@
 // depend on the routing), then reads all S = T*k expert ids (a few KB, served
 // from L2 after the first CTA) and builds in shared memory the histogram of all
 // entries and, in the same pass, the histogram of the entries that come before
-// token t.  With the exclusive scan of the (padded) counts, the slot of (t, j)
+// token t (shared-memory atomics).  With the exclusive scan of the (padded) counts, the slot of (t, j)
 // with expert e is
 //   offset[e] + before_t[e] + #{j' < j : topk_idx[t, j'] == e},
 // which is the stable (token, k) order.  The CTA then stores (or quantises and
@@ -102,13 +102,13 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_fused(FusedArgs 
                     raise_error(a.err, MOE_DEV_BAD_INDEX);
                 e = -1;
             }
-            const unsigned peers = __match_any_sync(kFullMask, e);
-            const unsigned below = __ballot_sync(kFullMask, i < mine);
-            if (e >= 0 && lane == (unsigned)(__ffs(peers) - 1)) {
-                atomicAdd(&hist[e], __popc(peers));
-                const int nb = __popc(peers & below);
-                if (nb)
-                    atomicAdd(&before[e], nb);
+            // Plain shared-memory atomics: at S <= kFusedMaxEntries a hot expert
+            // costs little, and grouping lanes first (match_any) cost more than
+            // it saved at decode sizes.
+            if (e >= 0) {
+                atomicAdd(&hist[e], 1);
+                if (i < mine)
+                    atomicAdd(&before[e], 1);
             }
         }
     }

@@ -212,6 +212,15 @@ def test_every_token_to_one_expert():
     check_problem(x, idx, w, E=8, R=2, fp8=False, pad128=True)
 
 
+def test_every_token_to_one_expert_fused_path():
+    # the one-launch kernel's shared-memory counters all hit one expert
+    T, k = 200, 2
+    x, _, w = random_problem(43, T, 512, 8, k)
+    idx = np.full((T, k), 6, np.int32)
+    idx[::3, 1] = 1
+    check_problem(x, idx, w, E=8, R=4, fp8=True, pad128=True)
+
+
 def test_zipf_routing_hot_expert_small_H():
     w, x, idx, wts = make_inputs("prefill_zipf", H=256)
     check_problem(x, idx, wts, E=w.E, R=w.R, fp8=True, pad128=False)
