@@ -275,7 +275,7 @@ int launch_layout(const moe_config *cfg, int32_t T, const int32_t *topk_idx,
 // register stores (and the fp8 quantiser) otherwise.
 int launch_payload(const moe_config *cfg, int32_t T, const void *x, const int32_t *slot,
                    const moe_dispatch_out *out, int32_t *dev_err, const DeviceInfo *dev,
-                   cudaStream_t s)
+                   cudaStream_t s, bool after_layout)
 {
     if (T == 0)
         return MOE_OK;
@@ -301,8 +301,12 @@ int launch_payload(const moe_config *cfg, int32_t T, const void *x, const int32_
         const int warps_per_cta = kScatterThreads / kWarp;
         const unsigned grid = grid_for((warp_units + warps_per_cta - 1) / warps_per_cta, dev->sms,
                                        2048 / kScatterThreads);
-        e = fp8 ? launch(scatter_rows<true>, grid, kScatterThreads, 0, s, a)
-                : launch(scatter_rows<false>, grid, kScatterThreads, 0, s, a);
+        if (after_layout)
+            e = fp8 ? launch(scatter_rows<true, true>, grid, kScatterThreads, 0, s, a)
+                    : launch(scatter_rows<false, true>, grid, kScatterThreads, 0, s, a);
+        else
+            e = fp8 ? launch(scatter_rows<true, false>, grid, kScatterThreads, 0, s, a)
+                    : launch(scatter_rows<false, false>, grid, kScatterThreads, 0, s, a);
     }
     return launched(e);
 }
@@ -416,7 +420,7 @@ int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
             return st;
     } else {
         if ((st = launch_layout(cfg, T, topk_idx, out, slot, workspace, dev_err, s)) != MOE_OK ||
-            (st = launch_payload(cfg, T, x, slot, out, dev_err, dev, s)) != MOE_OK)
+            (st = launch_payload(cfg, T, x, slot, out, dev_err, dev, s, true)) != MOE_OK)
             return st;
     }
     handle->cfg = *cfg;
@@ -457,7 +461,8 @@ int moe_dispatch_payload(const moe_config *cfg, int32_t T, const void *x, const 
     DeviceInfo *dev = nullptr;
     if ((st = device_info(&dev)) != MOE_OK)
         return st;
-    return launch_payload(cfg, T, x, slot, out, dev_err, dev, static_cast<cudaStream_t>(stream));
+    return launch_payload(cfg, T, x, slot, out, dev_err, dev, static_cast<cudaStream_t>(stream),
+                          false);
 }
 
 int moe_combine(const moe_handle *handle, const void *expert_out, void *y, int32_t *dev_err,

@@ -232,20 +232,29 @@ __device__ __forceinline__ void store_chunk(void *recv_x, float *recv_scale, int
     }
 }
 
-template <bool kFp8>
+// kEarlyLoad: the warp's first unit of x is loaded before waiting for the
+// previous kernel.  Only valid when the previous kernel in the stream is the
+// layout kernel of the same moe_dispatch call: that kernel waited for whatever
+// wrote x before it let this one launch, so x is complete in memory (and these
+// loads do not allocate in L1, so no stale line can exist).  Everything the
+// layout kernel writes (the slots) is read after the wait.
+template <bool kFp8, bool kEarlyLoad>
 __global__ void __launch_bounds__(kScatterThreads) scatter_rows(ScatterArgs a)
 {
-    stream_order_begin();
     constexpr int L = kScatterLaneCols;
     const int64_t nwarps = (int64_t)gridDim.x * (kScatterThreads / kWarp);
     const int32_t chunks = (a.H + chunk_cols<L>() - 1) / chunk_cols<L>();
     const int64_t units = (int64_t)a.T * chunks;
-    for (int64_t u = (int64_t)blockIdx.x * (kScatterThreads / kWarp) + threadIdx.x / kWarp;
-         u < units; u += nwarps) {
+    int64_t u = (int64_t)blockIdx.x * (kScatterThreads / kWarp) + threadIdx.x / kWarp;
+    LaneData<L> d;
+    if (kEarlyLoad && u < units)
+        load_chunk<L, kFp8>(a.x + (int64_t)(u / chunks) * a.H, a.H, (int32_t)(u % chunks), d);
+    stream_order_begin();
+    for (bool first = true; u < units; u += nwarps, first = false) {
         const int32_t t = (int32_t)(u / chunks);
         const int32_t c = (int32_t)(u % chunks);
-        LaneData<L> d;
-        load_chunk<L, kFp8>(a.x + (int64_t)t * a.H, a.H, c, d);
+        if (!(kEarlyLoad && first))
+            load_chunk<L, kFp8>(a.x + (int64_t)t * a.H, a.H, c, d);
         store_chunk<L, kFp8>(a.recv_x, a.recv_scale, a.H, c, a.k, a.slot + (int64_t)t * a.k,
                              a.rows_cap, a.err, d);
     }
@@ -328,8 +337,9 @@ __global__ void __launch_bounds__(kWarp) scatter_bulk_bf16(ScatterArgs a)
 }
 
 // Whether the bulk scatter applies: bf16 rows of at least 1 KB whose stages fit.
-// (fp8 stays on scatter_rows: its quantiser needs many warps per SM, and a
-// per-token barrier before the bulk stores cost more than they saved.)
+// fp8 stays on scatter_rows: three bulk-store designs for it (one warp
+// quantising per CTA, CTA-wide staging with a barrier per token, independent
+// warps with per-warp staging) all measured slower than register stores.
 inline bool use_bulk_scatter(int32_t H, bool fp8)
 {
     return !fp8 && H >= 512 && (uint64_t)kBulkStages * bulk_stage_bytes(H) <= kBulkMaxSmem;
