@@ -447,6 +447,107 @@ def run_gpu(args, rank, world):
                 set_bytes=set_bytes, l2=l2, per_graph=per_graph)
 
 
+# ---- the rows next to the hot path: one kernel at a time ---------------------------
+
+EXPERT_INTERMEDIATE = 2048  # DeepSeek-V3 / Kimi-K2 routed-expert intermediate size
+
+
+def run_op(args, peak, peak_kind):
+    """Times one next-row kernel on a workload's shapes; prints one JSON line."""
+    import math
+    import torch
+    import combine_route_meta_b200 as moe
+    from workloads import WORKLOADS, make_expert_out, make_inputs, normal_bf16_rows
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    _, x, idx, wts = make_inputs(w)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    stream = torch.cuda.Stream(device=dev)
+
+    def bf16_dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    d = moe.dispatch(bf16_dev(x), torch.from_numpy(idx).to(dev), torch.from_numpy(wts).to(dev),
+                     w.E, w.R, w.fp8, w.pad128)
+    rows = d.recv_x.shape[0]
+    S = w.T * w.k
+    if args.op == "rank_partial":
+        eo = bf16_dev(make_expert_out(w, rows))
+        set_bytes = rows * w.H * 2 + 2 * S * w.H * 2
+        make = lambda: dict(partial=torch.empty((w.T, w.k, w.H), dtype=torch.bfloat16, device=dev),
+                            prank=torch.empty((w.T, w.k), dtype=torch.int32, device=dev),
+                            npart=torch.empty(w.T, dtype=torch.int32, device=dev),
+                            y=torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev), eo=eo.clone())
+        fn = lambda b: (lambda: moe.combine_rank_partial_into(
+            d.handle.c, d.rank_offset, b["eo"], b["partial"], b["prank"], b["npart"], b["y"],
+            moe.error_word(dev), stream))
+    elif args.op == "silu_quant":
+        I = EXPERT_INTERMEDIATE
+        gu = bf16_dev(normal_bf16_rows(w.seed, 9, 0, rows, 2 * I))
+        set_bytes = rows * (4 * I + I + I // 32)
+        make = lambda: dict(gu=gu.clone(), act=torch.empty((rows, I), dtype=torch.float8_e4m3fn, device=dev),
+                            sc=torch.empty((rows, I // 128), dtype=torch.float32, device=dev))
+        fn = lambda b: (lambda: moe.silu_quant_into(b["gu"], d.recv_src, d.expert_offset[w.E:],
+                                                    b["act"], b["sc"], False, stream))
+    elif args.op == "router":
+        logits = torch.from_numpy(np.random.default_rng(w.seed).standard_normal((w.T, w.E)).astype(np.float32)).to(dev)
+        set_bytes = w.T * w.E * 4 + S * 8
+        make = lambda: dict(l=logits.clone(), idx=torch.empty((w.T, w.k), dtype=torch.int32, device=dev),
+                            w=torch.empty((w.T, w.k), dtype=torch.float32, device=dev))
+        fn = lambda b: (lambda: moe.router_topk_into(b["l"], w.k, b["idx"], b["w"],
+                                                     score_fn="sigmoid" if w.routing == "sigmoid_topk" else "softmax",
+                                                     stream=stream))
+    else:
+        raise SystemExit(f"unknown --op {args.op}")
+    nsets = 1 if set_bytes >= 2 * l2 else min(64, math.ceil(2 * l2 / set_bytes) + 1)
+    sets = [make() for _ in range(nsets)]
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for b in sets:
+            fn(b)()
+    stream.synchronize()
+    per_graph = max(nsets, 8)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(per_graph):
+            fn(sets[i % nsets])()
+    reps = max(1, args.steps // per_graph)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for timed in (False, True):
+        with torch.cuda.stream(stream):
+            torch.cuda._sleep(min(reps, 256) * 100_000)
+            e0.record(stream)
+            for _ in range(reps if timed else max(1, args.warmup // per_graph)):
+                g.replay()
+            e1.record(stream)
+        e1.synchronize()
+    launches = reps * per_graph
+    us = e0.elapsed_time(e1) * 1e3 / launches
+    if moe.check(stream):
+        raise RuntimeError("device error bits during timing")
+    # algorithmic bytes of one launch
+    if args.op == "rank_partial":
+        npart = int(sets[0]["npart"].sum().item())
+        nbytes = S * w.H * 2 + 2 * S * 4 + (w.R + 1) * 4 + 2 * npart * w.H * 2 + w.T * 4 + w.T * w.H * 2
+        extra = {"partials": npart}
+    elif args.op == "silu_quant":
+        used = int((d.recv_src >= 0).sum().item())
+        I = EXPERT_INTERMEDIATE
+        nbytes = used * (4 * I + I + (I // 128) * 4) + used * 4
+        extra = {"rows_used": used, "I": I}
+    else:
+        nbytes = w.T * w.E * 4 + S * 8
+        extra = {}
+    gbs = nbytes / (us * 1e-6) / 1e9
+    line = {"op": args.op, "workload": w.name, "us": round(us, 3), "algorithmic_bytes": nbytes,
+            "achieved_GBs": round(gbs, 1), "peak": peak, "peak_kind": peak_kind,
+            "frac": round(gbs / peak, 4), "launches_timed": launches,
+            "l2": f"{nsets} rotating sets of {set_bytes / 1e6:.1f} MB", **extra}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -455,6 +556,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", default=None, choices=["rank_partial", "silu_quant", "router"],
+                    help="time one of the kernels next to the hot path instead of the step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -464,6 +567,10 @@ def main():
     from workloads import WORKLOADS
     w0 = WORKLOADS[args.workload]
     peak, peak_kind = measured_peak()
+
+    if args.op is not None:
+        run_op(args, peak, peak_kind)
+        return
 
     if args.impl == "reference":
         # The reference arm is the CPU oracle, timed on this host's cores (rank 0 only).

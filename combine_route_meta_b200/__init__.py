@@ -51,6 +51,8 @@ DEV_BAD_SLOT = 8
 
 MAX_EXPERTS = 2048
 MAX_TOPK = 64
+SCORE_SOFTMAX = 0
+SCORE_SIGMOID = 1
 NO_ALLOC_SCRATCH_BYTES = 1 << 20
 
 
@@ -101,6 +103,12 @@ def _declare(lib):
     lib.moe_combine.restype = ctypes.c_int
     lib.moe_selftest_bounded_wait.argtypes = [P, ctypes.c_uint64, P]
     lib.moe_selftest_bounded_wait.restype = ctypes.c_int
+    lib.moe_combine_rank_partial.argtypes = [ctypes.POINTER(moe_handle), P, P, P, P, P, P, P, P]
+    lib.moe_combine_rank_partial.restype = ctypes.c_int
+    lib.moe_silu_quant.argtypes = [i64, i32, P, P, P, P, P, i32, P]
+    lib.moe_silu_quant.restype = ctypes.c_int
+    lib.moe_router_topk.argtypes = [i32, i32, i32, P, i32, i32, i32, i32, P, P, P]
+    lib.moe_router_topk.restype = ctypes.c_int
     lib.moe_check.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
     lib.moe_check.restype = ctypes.c_int
     return lib
@@ -121,6 +129,9 @@ moe_dispatch_payload = lib.moe_dispatch_payload
 moe_combine = lib.moe_combine
 moe_check = lib.moe_check
 moe_selftest_bounded_wait = lib.moe_selftest_bounded_wait
+moe_combine_rank_partial = lib.moe_combine_rank_partial
+moe_silu_quant = lib.moe_silu_quant
+moe_router_topk = lib.moe_router_topk
 
 
 class MoeError(RuntimeError):
@@ -320,3 +331,76 @@ def combine(handle: Handle, expert_out: torch.Tensor, *,
     y = torch.empty((c.T, c.cfg.H), dtype=torch.bfloat16, device=expert_out.device)
     combine_into(c, expert_out, y, error_word(expert_out.device), stream)
     return y
+
+
+def combine_rank_partial_into(handle_c: moe_handle, rank_offset: torch.Tensor,
+                              expert_out: torch.Tensor, partial: torch.Tensor,
+                              partial_rank: torch.Tensor, npart: torch.Tensor, y: torch.Tensor,
+                              err: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> None:
+    """moe_combine_rank_partial into preallocated buffers."""
+    P = ctypes.c_void_p
+    st = lib.moe_combine_rank_partial(ctypes.byref(handle_c), P(rank_offset.data_ptr()),
+                                      P(expert_out.data_ptr()), P(partial.data_ptr()),
+                                      P(partial_rank.data_ptr()), P(npart.data_ptr()),
+                                      P(y.data_ptr()), P(err.data_ptr()), P(_stream_ptr(stream)))
+    _ok(st, "moe_combine_rank_partial")
+
+
+def combine_rank_partial(handle: Handle, rank_offset: torch.Tensor, expert_out: torch.Tensor, *,
+                         stream: Optional[torch.cuda.Stream] = None):
+    """(y, partial, partial_rank, npart): combine with per-rank partial sums (see the C header)."""
+    c = handle.c
+    dev = expert_out.device
+    partial = torch.empty((c.T, c.cfg.k, c.cfg.H), dtype=torch.bfloat16, device=dev)
+    partial_rank = torch.full((c.T, c.cfg.k), -1, dtype=torch.int32, device=dev)
+    npart = torch.empty(c.T, dtype=torch.int32, device=dev)
+    y = torch.empty((c.T, c.cfg.H), dtype=torch.bfloat16, device=dev)
+    combine_rank_partial_into(c, rank_offset, expert_out, partial, partial_rank, npart, y,
+                              error_word(dev), stream)
+    return y, partial, partial_rank, npart
+
+
+def silu_quant_into(gate_up: torch.Tensor, recv_src: torch.Tensor, rows_in_use: torch.Tensor,
+                    act: torch.Tensor, act_scale: torch.Tensor, col_major: bool = False,
+                    stream: Optional[torch.cuda.Stream] = None) -> None:
+    """moe_silu_quant into preallocated act (float8_e4m3fn) and act_scale (float32)."""
+    P = ctypes.c_void_p
+    rows_cap, two_i = gate_up.shape
+    st = lib.moe_silu_quant(rows_cap, two_i // 2, P(gate_up.data_ptr()), P(recv_src.data_ptr()),
+                            P(rows_in_use.data_ptr()), P(act.data_ptr()), P(act_scale.data_ptr()),
+                            1 if col_major else 0, P(_stream_ptr(stream)))
+    _ok(st, "moe_silu_quant")
+
+
+def silu_quant(gate_up: torch.Tensor, recv_src: torch.Tensor, rows_in_use: torch.Tensor, *,
+               col_major: bool = False, stream: Optional[torch.cuda.Stream] = None):
+    """(act, act_scale): block-fp8 SiLU(gate) * up of the populated rows (see the C header)."""
+    rows_cap, two_i = gate_up.shape
+    I = two_i // 2
+    act = torch.zeros((rows_cap, I), dtype=torch.float8_e4m3fn, device=gate_up.device)
+    shape = (I // 128, rows_cap) if col_major else (rows_cap, I // 128)
+    act_scale = torch.zeros(shape, dtype=torch.float32, device=gate_up.device)
+    silu_quant_into(gate_up, recv_src, rows_in_use, act, act_scale, col_major, stream)
+    return act, act_scale
+
+
+def router_topk_into(logits: torch.Tensor, k: int, topk_idx: torch.Tensor, topk_w: torch.Tensor, *,
+                     score_fn: str = "softmax", n_group: int = 1, topk_group: int = 1,
+                     renormalize: bool = True, stream: Optional[torch.cuda.Stream] = None) -> None:
+    """moe_router_topk into preallocated topk_idx (int32) and topk_w (float32)."""
+    T, E = logits.shape
+    P = ctypes.c_void_p
+    st = lib.moe_router_topk(T, E, k, P(logits.data_ptr()),
+                             {"softmax": SCORE_SOFTMAX, "sigmoid": SCORE_SIGMOID}[score_fn],
+                             n_group, topk_group, 1 if renormalize else 0,
+                             P(topk_idx.data_ptr()), P(topk_w.data_ptr()), P(_stream_ptr(stream)))
+    _ok(st, "moe_router_topk")
+
+
+def router_topk(logits: torch.Tensor, k: int, **kw):
+    """(topk_idx, topk_w) of group-limited top-k routing (see the C header)."""
+    T = logits.shape[0]
+    idx = torch.empty((T, k), dtype=torch.int32, device=logits.device)
+    w = torch.empty((T, k), dtype=torch.float32, device=logits.device)
+    router_topk_into(logits.contiguous().float(), k, idx, w, **kw)
+    return idx, w

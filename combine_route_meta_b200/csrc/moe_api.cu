@@ -10,10 +10,13 @@
 #include "moe_dispatch_combine.h"
 
 #include "combine.cuh"
+#include "combine_partial.cuh"
 #include "common.cuh"
 #include "dispatch_fused.cuh"
 #include "meta.cuh"
+#include "router.cuh"
 #include "scatter.cuh"
+#include "silu_quant.cuh"
 
 // Scratch of moe_dispatch_no_alloc: a fixed array in device memory, allocated
 // by the CUDA runtime when the library's module is loaded on a device and held
@@ -529,6 +532,119 @@ int moe_selftest_bounded_wait(int32_t *dev_err, uint64_t limit_ns, void *stream)
         return MOE_ERR_INVALID_ARG;
     return launched(launch(wait_selftest, 1, kWarp, 0, static_cast<cudaStream_t>(stream), dev_err,
                            limit_ns));
+}
+
+int moe_combine_rank_partial(const moe_handle *handle, const int32_t *rank_offset,
+                             const void *expert_out, void *partial, int32_t *partial_rank,
+                             int32_t *npart, void *y, int32_t *dev_err, void *stream)
+{
+    if (handle == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    int st = check_config(&handle->cfg);
+    if (st != MOE_OK)
+        return st;
+    const moe_config &c = handle->cfg;
+    if (handle->T < 0 || handle->rows_cap < 0)
+        return MOE_ERR_INVALID_ARG;
+    if (handle->T == 0)
+        return MOE_OK;
+    if (handle->slot == nullptr || handle->topk_w == nullptr || rank_offset == nullptr ||
+        partial == nullptr || partial_rank == nullptr || npart == nullptr || y == nullptr ||
+        (handle->rows_cap > 0 && expert_out == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(expert_out) || !aligned16(partial) || !aligned16(y))
+        return MOE_ERR_INVALID_ARG;
+    DeviceInfo *dev = nullptr;
+    if ((st = device_info(&dev)) != MOE_OK)
+        return st;
+    PartialArgs a;
+    a.expert_out = static_cast<const uint16_t *>(expert_out);
+    a.slot = handle->slot;
+    a.w = handle->topk_w;
+    a.rank_offset = rank_offset;
+    a.T = handle->T;
+    a.H = c.H;
+    a.k = c.k;
+    a.R = c.R;
+    a.parts = (c.H / 8 + kPartialThreads - 1) / kPartialThreads;
+    a.rows_cap = handle->rows_cap;
+    a.partial = static_cast<uint16_t *>(partial);
+    a.partial_rank = partial_rank;
+    a.npart = npart;
+    a.y = static_cast<uint16_t *>(y);
+    a.err = dev_err;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const unsigned grid = grid_for((int64_t)a.T * a.parts, dev->sms, 16);
+    if ((st = launched(launch(combine_partial_send, grid, kPartialThreads, 0, s, a))) != MOE_OK)
+        return st;
+    return launched(launch(combine_partial_recv, grid, kPartialThreads, 0, s, a));
+}
+
+int moe_silu_quant(int64_t rows_cap, int32_t I, const void *gate_up, const int32_t *recv_src,
+                   const int32_t *rows_in_use, void *act, float *act_scale,
+                   int32_t scale_col_major, void *stream)
+{
+    if (rows_cap < 0 || rows_cap > INT32_MAX || I <= 0)
+        return MOE_ERR_INVALID_ARG;
+    if (I % 128 != 0)
+        return MOE_ERR_UNSUPPORTED;
+    if (rows_cap == 0)
+        return MOE_OK;
+    if (gate_up == nullptr || recv_src == nullptr || rows_in_use == nullptr || act == nullptr ||
+        act_scale == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(gate_up) || !aligned16(act))
+        return MOE_ERR_INVALID_ARG;
+    DeviceInfo *dev = nullptr;
+    int st;
+    if ((st = device_info(&dev)) != MOE_OK)
+        return st;
+    SiluQuantArgs a;
+    a.gate_up = static_cast<const uint16_t *>(gate_up);
+    a.recv_src = recv_src;
+    a.rows_in_use = rows_in_use;
+    a.rows_cap = rows_cap;
+    a.I = I;
+    a.act = static_cast<uint8_t *>(act);
+    a.scale = act_scale;
+    a.col_major = scale_col_major ? 1 : 0;
+    // A fixed grid, whatever the routing: the kernel reads how many rows are in use.
+    const unsigned grid = (unsigned)(dev->sms * kSiluCtasPerSm);
+    return launched(launch(silu_quant_rows, grid, kSiluThreads, 0, static_cast<cudaStream_t>(stream), a));
+}
+
+int moe_router_topk(int32_t T, int32_t E, int32_t k, const float *logits, int32_t score_fn,
+                    int32_t n_group, int32_t topk_group, int32_t renormalize, int32_t *topk_idx,
+                    float *topk_w, void *stream)
+{
+    if (T < 0 || E <= 0 || k <= 0 || n_group <= 0 || topk_group <= 0 || topk_group > n_group ||
+        (score_fn != MOE_SCORE_SOFTMAX && score_fn != MOE_SCORE_SIGMOID) || E % n_group != 0)
+        return MOE_ERR_INVALID_ARG;
+    if ((int64_t)k > (int64_t)topk_group * (E / n_group))
+        return MOE_ERR_INVALID_ARG;
+    if (E > kRouterMaxE || k > kRouterMaxK || n_group > kRouterMaxGroups)
+        return MOE_ERR_UNSUPPORTED;
+    if (T == 0)
+        return MOE_OK;
+    if (logits == nullptr || topk_idx == nullptr || topk_w == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    DeviceInfo *dev = nullptr;
+    int st;
+    if ((st = device_info(&dev)) != MOE_OK)
+        return st;
+    RouterArgs a;
+    a.logits = logits;
+    a.T = T;
+    a.E = E;
+    a.k = k;
+    a.score_fn = score_fn;
+    a.n_group = n_group;
+    a.topk_group = topk_group;
+    a.renormalize = renormalize ? 1 : 0;
+    a.topk_idx = topk_idx;
+    a.topk_w = topk_w;
+    const unsigned grid = grid_for((T + kRouterWarps - 1) / kRouterWarps, dev->sms, 16);
+    return launched(launch(router_topk, grid, kRouterWarps * kWarp, 0, static_cast<cudaStream_t>(stream), a));
 }
 
 int moe_check(int32_t *dev_err, void *stream, int32_t *bits_out)

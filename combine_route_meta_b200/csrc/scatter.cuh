@@ -90,27 +90,17 @@ __device__ __forceinline__ float quotient_for_e4m3(float x, float scale, float r
 // e4m3 codes of the lane's values, element 0 in the lowest byte, and the scale
 // of the lane's 128-column block.  All lanes of the warp call this together
 // (inactive lanes hold zeros).
+// e4m3 codes and the block scale of kLaneCols binary32 values per lane; the
+// 128/kLaneCols lanes of a 128-column block reduce the maximum together (all
+// lanes of the warp call this).
 template <int kLaneCols>
-__device__ __forceinline__ void quantise_lane(const LaneData<kLaneCols> &d, uint32_t (&codes)[kLaneCols / 4],
-                                              float &scale_out)
+__device__ __forceinline__ void quantise_floats(const float (&f)[kLaneCols],
+                                                uint32_t (&codes)[kLaneCols / 4], float &scale_out)
 {
-    float f[kLaneCols];
-#pragma unroll
-    for (int i = 0; i < kLaneCols / 8; ++i) {
-        f[8 * i + 0] = bf16_lo(d.v[i].x);
-        f[8 * i + 1] = bf16_hi(d.v[i].x);
-        f[8 * i + 2] = bf16_lo(d.v[i].y);
-        f[8 * i + 3] = bf16_hi(d.v[i].y);
-        f[8 * i + 4] = bf16_lo(d.v[i].z);
-        f[8 * i + 5] = bf16_hi(d.v[i].z);
-        f[8 * i + 6] = bf16_lo(d.v[i].w);
-        f[8 * i + 7] = bf16_hi(d.v[i].w);
-    }
     float amax = 0.0f;
 #pragma unroll
     for (int i = 0; i < kLaneCols; ++i)
         amax = fmaxf(amax, fabsf(f[i]));
-    // butterfly over the 128/kLaneCols lanes of the block
 #pragma unroll
     for (int d = 64 / kLaneCols; d >= 1; d >>= 1)
         amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, d));
@@ -132,6 +122,25 @@ __device__ __forceinline__ void quantise_lane(const LaneData<kLaneCols> &d, uint
         }
     }
     scale_out = scale;
+}
+
+template <int kLaneCols>
+__device__ __forceinline__ void quantise_lane(const LaneData<kLaneCols> &d, uint32_t (&codes)[kLaneCols / 4],
+                                              float &scale_out)
+{
+    float f[kLaneCols];
+#pragma unroll
+    for (int i = 0; i < kLaneCols / 8; ++i) {
+        f[8 * i + 0] = bf16_lo(d.v[i].x);
+        f[8 * i + 1] = bf16_hi(d.v[i].x);
+        f[8 * i + 2] = bf16_lo(d.v[i].y);
+        f[8 * i + 3] = bf16_hi(d.v[i].y);
+        f[8 * i + 4] = bf16_lo(d.v[i].z);
+        f[8 * i + 5] = bf16_hi(d.v[i].z);
+        f[8 * i + 6] = bf16_lo(d.v[i].w);
+        f[8 * i + 7] = bf16_hi(d.v[i].w);
+    }
+    quantise_floats<kLaneCols>(f, codes, scale_out);
 }
 
 // First column of the lane's vector i in chunk c.

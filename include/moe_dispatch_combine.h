@@ -73,6 +73,10 @@ extern "C" {
 #define MOE_DEV_TIMEOUT 4   /* a bounded device wait (1 s) gave up                     */
 #define MOE_DEV_BAD_SLOT 8  /* payload / combine: a slot outside [-1, rows_cap)        */
 
+/* Router score functions (moe_router_topk). */
+#define MOE_SCORE_SOFTMAX 0
+#define MOE_SCORE_SIGMOID 1
+
 /* Limits of this build. */
 #define MOE_MAX_EXPERTS 2048 /* E */
 #define MOE_MAX_TOPK 64      /* k */
@@ -225,6 +229,83 @@ MOE_API int moe_dispatch_payload(const moe_config *cfg, int32_t T, const void *x
  */
 MOE_API int moe_combine(const moe_handle *handle, const void *expert_out, void *y, int32_t *dev_err,
                 void *stream);
+
+/*
+ * Combine with sender-side (per-rank) partial accumulation ("Enabling
+ * trillion-parameter models on AWS EFA", section "Avaliação": DeepEP
+ * accumulates on the sending side to move less data, which may change
+ * precision).  Same inputs as moe_combine plus the dispatch's rank_offset.
+ *
+ *   1. send: for each token t and each distinct rank r_q among the ranks of
+ *      t's kept entries (q in order of first appearance over j; the rank of a
+ *      receive row s is the r with rank_offset[r] <= s < rank_offset[r+1]):
+ *        partial[t, q, :] = bf16( sum over t's entries j on rank r_q, ascending
+ *                                 j, of an fp32 fma of topk_w[t,j] * row )
+ *      partial_rank[t, q] = r_q, npart[t] = number of distinct ranks.
+ *   2. receive: y[t, :] = bf16( sum_{q < npart[t]} partial[t, q, :] ) in fp32.
+ *
+ *   rank_offset   [R+1] int32 device (from moe_dispatch).
+ *   partial       [T, k, H] bf16 device, 16-byte aligned (the "send buffer";
+ *                 rows q >= npart[t] are not written).
+ *   partial_rank  [T, k] int32 device;  npart [T] int32 device.
+ *   y             [T, H] bf16 device, 16-byte aligned.
+ * Compared with moe_combine, each partial is rounded to bf16 once more.
+ * Returns MOE_OK or a negative status.
+ */
+MOE_API int moe_combine_rank_partial(const moe_handle *handle, const int32_t *rank_offset,
+                                     const void *expert_out, void *partial,
+                                     int32_t *partial_rank, int32_t *npart, void *y,
+                                     int32_t *dev_err, void *stream);
+
+/*
+ * Expert-side activation: act = e4m3 block quantisation of SiLU(gate) * up
+ * ("Lower latency and higher throughput with multi-node DeepSeek deployment",
+ * section "Quantização": the SiLU kernel emits block-fp8 activations for the
+ * next grouped GEMM and, to stay valid under CUDA graphs with data-dependent
+ * routing, runs a fixed set of persistent workers that read how many rows the
+ * routing populated).
+ *
+ *   gate_up      [rows_cap, 2I] bf16 device, 16-byte aligned: gate in columns
+ *                [0, I), up in [I, 2I), in a dispatch's receive layout.
+ *   recv_src     [rows_cap] int32 device (from moe_dispatch): rows with -1 are
+ *                padding and are skipped.
+ *   rows_in_use  device int32: rows at or past it are skipped (normally
+ *                &expert_offset[E]); clamped to [0, rows_cap].
+ *   act          [rows_cap, I] e4m3 bytes device, 16-byte aligned.
+ *   act_scale    fp32 device: [rows_cap, I/128] row-major, or with
+ *                scale_col_major != 0, [I/128, rows_cap] (one column of scales
+ *                per row, the layout grouped GEMMs read).
+ * SiLU(g) = g / (1 + e^-g) in binary32, with e^x by Cody-Waite reduction and a
+ * degree-7 Taylor polynomial (fused multiply-adds), -0 below g = -88; the
+ * activation is the binary32 product with up.  Per 128 columns: scale =
+ * amax/448, codes = e4m3(a/scale) as in moe_dispatch.  I must be a multiple of
+ * 128 (else MOE_ERR_UNSUPPORTED).  Rows not selected are left untouched.
+ */
+MOE_API int moe_silu_quant(int64_t rows_cap, int32_t I, const void *gate_up,
+                           const int32_t *recv_src, const int32_t *rows_in_use, void *act,
+                           float *act_scale, int32_t scale_col_major, void *stream);
+
+/*
+ * Router top-k ("Lower latency and higher throughput with multi-node DeepSeek
+ * deployment", section "Roteador MoE": one top-k with index tracking serves all
+ * MoE models; plain top-k is group-limited top-k with one group).  For each
+ * token's logits[t, 0..E) (fp32 device):
+ *   - the experts form n_group contiguous groups of E/n_group; a group's score
+ *     is its largest logit; the topk_group best groups are kept (ties: lower
+ *     group id);
+ *   - the k largest logits among the kept groups' experts are chosen, best
+ *     first (ties: lower expert id) -> topk_idx[t, 0..k) (int32 device);
+ *   - topk_w[t, j] (fp32 device): MOE_SCORE_SOFTMAX: exp(l_j - m) divided by
+ *     the sum over the k chosen (renormalize != 0) or over all E logits;
+ *     MOE_SCORE_SIGMOID: 1/(1+exp(-l_j)), divided by the chosen ones' sum when
+ *     renormalize != 0.
+ * The choice compares logits only (both score functions are increasing), so
+ * it is exact.  Limits: E <= 1024, k <= 32, n_group <= 32, E % n_group == 0,
+ * k <= topk_group * E / n_group.  Returns a status.
+ */
+MOE_API int moe_router_topk(int32_t T, int32_t E, int32_t k, const float *logits,
+                            int32_t score_fn, int32_t n_group, int32_t topk_group,
+                            int32_t renormalize, int32_t *topk_idx, float *topk_w, void *stream);
 
 /*
  * moe_dispatch without a workspace argument, for callers that cannot allocate

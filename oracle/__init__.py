@@ -56,6 +56,14 @@ def _load():
         lib.oracle_dispatch.restype = i32
         lib.oracle_combine.argtypes = [i32, i32, i32, P, P, P, P]
         lib.oracle_combine.restype = None
+        lib.oracle_combine_rank_partial.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P]
+        lib.oracle_combine_rank_partial.restype = None
+        lib.oracle_silu_f32.argtypes = [ctypes.c_float]
+        lib.oracle_silu_f32.restype = ctypes.c_float
+        lib.oracle_silu_quant.argtypes = [i64, i32, P, P, i64, P, P, i32]
+        lib.oracle_silu_quant.restype = None
+        lib.oracle_router_topk.argtypes = [i32, i32, i32, P, i32, i32, i32, i32, P, P]
+        lib.oracle_router_topk.restype = None
         lib.oracle_quantise_row_fp8.argtypes = [P, i32, P, P]
         lib.oracle_quantise_row_fp8.restype = None
         _lib = lib
@@ -168,3 +176,60 @@ def combine(slot, topk_w, expert_out_bf16, tokens=None) -> np.ndarray:
     y = np.zeros((T, H), np.float64)
     _load().oracle_combine(T, H, k, _ptr(slot), _ptr(w), _ptr(eo), _ptr(y))
     return y
+
+
+def combine_rank_partial(topk_idx, slot, topk_w, expert_out_bf16, *, E: int, R: int):
+    """Sender-side (per-rank) partial combine.  Returns dict with partial
+    (uint16 [T,k,H], bf16 bits), partial_rank [T,k], npart [T], y (fp64 [T,H])."""
+    idx = _c(topk_idx, np.int32)
+    slot = _c(slot, np.int32)
+    w = _c(topk_w, np.float32)
+    eo = _c(expert_out_bf16, np.uint16)
+    T = slot.shape[0]
+    k = slot.shape[1] if slot.ndim == 2 else 0
+    H = eo.shape[1]
+    out = dict(partial=np.zeros((T, k, H), np.uint16), partial_rank=np.full((T, k), -1, np.int32),
+               npart=np.zeros(T, np.int32), y=np.zeros((T, H), np.float64))
+    _load().oracle_combine_rank_partial(T, H, k, E, R, _ptr(idx), _ptr(slot), _ptr(w), _ptr(eo),
+                                        _ptr(out["partial"]), _ptr(out["partial_rank"]),
+                                        _ptr(out["npart"]), _ptr(out["y"]))
+    return out
+
+
+def silu_f32(g: float) -> float:
+    """SiLU in binary32 as the oracle defines it (see moe_oracle.c)."""
+    return float(_load().oracle_silu_f32(float(np.float32(g))))
+
+
+def silu_quant(gate_up_bf16, recv_src, rows_in_use: int, *, col_major: bool = False,
+               fill: int = 0):
+    """(act uint8 [rows_cap, I], scale float32) of the expert-side SiLU + block quantiser.
+    Rows that are not written keep `fill` bytes."""
+    gu = _c(gate_up_bf16, np.uint16)
+    src = _c(recv_src, np.int32)
+    rows_cap, two_i = gu.shape
+    I = two_i // 2
+    if I % 128:
+        raise ValueError("I must be a multiple of 128")
+    act = np.full((rows_cap, I), fill, np.uint8)
+    shape = (I // 128, rows_cap) if col_major else (rows_cap, I // 128)
+    scale = np.zeros(shape, np.float32)
+    if fill:
+        scale.view(np.uint8)[:] = fill
+    _load().oracle_silu_quant(rows_cap, I, _ptr(gu), _ptr(src), int(rows_in_use), _ptr(act),
+                              _ptr(scale), int(bool(col_major)))
+    return act, scale
+
+
+def router_topk(logits, k: int, *, score_fn: str = "softmax", n_group: int = 1,
+                topk_group: int = 1, renormalize: bool = True):
+    """(topk_idx int32 [T,k], topk_w float32 [T,k]) of group-limited top-k routing."""
+    l = _c(logits, np.float32)
+    T, E = l.shape
+    if k > 64 or E % n_group or not (1 <= topk_group <= n_group) or k > topk_group * (E // n_group):
+        raise ValueError("unsupported router shape")
+    idx = np.zeros((T, k), np.int32)
+    w = np.zeros((T, k), np.float32)
+    _load().oracle_router_topk(T, E, k, _ptr(l), {"softmax": 0, "sigmoid": 1}[score_fn], n_group,
+                               topk_group, int(bool(renormalize)), _ptr(idx), _ptr(w))
+    return idx, w

@@ -254,3 +254,265 @@ void oracle_quantise_row_fp8(const uint16_t *x, int32_t H, uint8_t *codes, float
 {
     quantise_row_fp8(x, H, codes, scales);
 }
+
+/* The nearest bf16 (8 significant bits, ties to even) to a double, rounded
+ * once and directly, as bf16 bits.  Inputs here are finite and far from the
+ * bf16 range limits. */
+static uint16_t double_to_bf16(double v)
+{
+    if (v == 0.0)
+        return signbit(v) ? 0x8000 : 0x0000;
+    int e;
+    double f = frexp(fabs(v), &e); /* |v| = f * 2^e, f in [0.5, 1) */
+    /* 8 significant bits: units of 2^(e-8) */
+    double units = nearbyint(ldexp(f, 8));
+    double q = ldexp(units, e - 8);
+    float qf = (float)q; /* exact: q has at most 9 significant bits */
+    uint32_t u;
+    memcpy(&u, &qf, sizeof u);
+    uint16_t b = (uint16_t)(u >> 16);
+    return (uint16_t)(signbit(v) ? (b | 0x8000) : b);
+}
+
+/*
+ * Sender-side (per-rank) partial accumulation of combine.  "Enabling
+ * trillion-parameter models on AWS EFA", section "Avaliação": DeepEP
+ * accumulates on the sending side to move less data, which may change
+ * precision.  Each rank r sums, for token t, the weighted rows of t's entries
+ * whose experts it hosts (rank of expert e: e / (E/R)), and sends that partial
+ * as one bf16 row; the token's home then sums the partials.
+ *
+ * Outputs: partial[t, q, :] (bf16 bits, q-th distinct rank of token t in order
+ * of first appearance over j), partial_rank[t, q], npart[t]; and y[t, :] =
+ * sum_q partial[t, q] (fp64).  Entries with slot -1 are skipped; a token with
+ * no kept entry has npart 0 and y 0.
+ */
+void oracle_combine_rank_partial(int32_t T, int32_t H, int32_t k, int32_t E, int32_t R,
+                                 const int32_t *topk_idx, const int32_t *slot,
+                                 const float *topk_w, const uint16_t *expert_out,
+                                 uint16_t *partial, int32_t *partial_rank, int32_t *npart,
+                                 double *y)
+{
+    const int32_t per_rank = E / R;
+    double *acc = (double *)malloc(sizeof(double) * (size_t)(H > 0 ? H : 1));
+    for (int32_t t = 0; t < T; ++t) {
+        int32_t n = 0;
+        for (int32_t j = 0; j < k; ++j) {
+            int32_t s = slot[(int64_t)t * k + j];
+            if (s < 0)
+                continue;
+            int32_t r = topk_idx[(int64_t)t * k + j] / per_rank;
+            int seen = 0;
+            for (int32_t q = 0; q < n; ++q)
+                if (partial_rank[(int64_t)t * k + q] == r)
+                    seen = 1;
+            if (seen)
+                continue; /* this rank's partial was formed at its first entry */
+            for (int32_t h = 0; h < H; ++h)
+                acc[h] = 0.0;
+            for (int32_t jj = j; jj < k; ++jj) {
+                int32_t s2 = slot[(int64_t)t * k + jj];
+                if (s2 < 0 || topk_idx[(int64_t)t * k + jj] / per_rank != r)
+                    continue;
+                for (int32_t h = 0; h < H; ++h)
+                    acc[h] += (double)topk_w[(int64_t)t * k + jj] *
+                              (double)bf16_to_float(expert_out[(int64_t)s2 * H + h]);
+            }
+            for (int32_t h = 0; h < H; ++h)
+                partial[((int64_t)t * k + n) * H + h] = double_to_bf16(acc[h]);
+            partial_rank[(int64_t)t * k + n] = r;
+            ++n;
+        }
+        npart[t] = n;
+        for (int32_t h = 0; h < H; ++h) {
+            double sum = 0.0;
+            for (int32_t q = 0; q < n; ++q)
+                sum += (double)bf16_to_float(partial[((int64_t)t * k + q) * H + h]);
+            y[(int64_t)t * H + h] = sum;
+        }
+    }
+    free(acc);
+}
+
+/*
+ * e^x in binary32 for x in [-87, 88], by Cody-Waite argument reduction and a
+ * degree-7 Taylor polynomial (Cody and Waite, "Software Manual for the
+ * Elementary Functions", 1980): x = n*ln2 + r with n = rint(x*log2(e)) and
+ * |r| <= ln2/2, r computed with ln2 split in a high part (exact products) and a
+ * low part; e^r = sum_{i<=7} r^i/i! by Horner's rule with fused multiply-adds;
+ * then scaled by 2^n.  Every step is one IEEE operation, so the value is a
+ * fixed function of x.
+ */
+static float exp_cody_waite(float x)
+{
+    const float n = rintf(x * 1.44269504088896341f);
+    float r = fmaf(-n, 0.693145751953125f, x);
+    r = fmaf(-n, 1.42860682030941723212e-6f, r);
+    float p = 1.98412698412698413e-4f; /* 1/7! */
+    p = fmaf(p, r, 1.38888888888888889e-3f); /* 1/6! */
+    p = fmaf(p, r, 8.33333333333333333e-3f); /* 1/5! */
+    p = fmaf(p, r, 4.16666666666666667e-2f); /* 1/4! */
+    p = fmaf(p, r, 1.66666666666666667e-1f); /* 1/3! */
+    p = fmaf(p, r, 0.5f);
+    p = fmaf(p, r, 1.0f);
+    p = fmaf(p, r, 1.0f);
+    /* 2^n, n in [-126, 127], from its exponent bits */
+    const uint32_t bits = (uint32_t)((int32_t)n + 127) << 23;
+    float two_n;
+    memcpy(&two_n, &bits, sizeof two_n);
+    return p * two_n;
+}
+
+/* SiLU in binary32: g / (1 + e^-g).  Below g = -88 the result is -0 (the true
+ * magnitude is under 5.3e-37); above g = 87, 1 + e^-g rounds to 1, so the
+ * exponent argument is clamped at -87 without changing the result. */
+float oracle_silu_f32(float g)
+{
+    if (g < -88.0f)
+        return -0.0f;
+    float x = -g;
+    if (x < -87.0f)
+        x = -87.0f;
+    return g / (1.0f + exp_cody_waite(x));
+}
+
+/*
+ * Expert-side activation and block quantiser ("Lower latency and higher
+ * throughput with multi-node DeepSeek deployment", section "Quantização": the
+ * SiLU kernel splits activations along the hidden dimension and takes the
+ * largest magnitude of every 128-element block for its scale; it reads the
+ * routing counts to know which rows are populated).
+ *   gate_up [rows_cap, 2I] bf16: gate = columns [0, I), up = [I, 2I).
+ *   a = silu(gate) * up (binary32), then per 128-block: scale = amax/448,
+ *   codes e4m3(a/scale) as in the dispatch quantiser.
+ * Only rows r < rows_in_use with recv_src[r] >= 0 are written.  Scales are
+ * row-major [rows_cap, I/128] or, with col_major, [I/128, rows_cap].
+ */
+void oracle_silu_quant(int64_t rows_cap, int32_t I, const uint16_t *gate_up,
+                       const int32_t *recv_src, int64_t rows_in_use, uint8_t *act,
+                       float *act_scale, int32_t col_major)
+{
+    const int32_t nb = I / 128;
+    float *a = (float *)malloc(sizeof(float) * (size_t)(I > 0 ? I : 1));
+    if (rows_in_use > rows_cap)
+        rows_in_use = rows_cap;
+    for (int64_t r = 0; r < rows_in_use; ++r) {
+        if (recv_src[r] < 0)
+            continue;
+        const uint16_t *g = gate_up + r * 2 * (int64_t)I;
+        const uint16_t *u = g + I;
+        for (int32_t i = 0; i < I; ++i)
+            a[i] = oracle_silu_f32(bf16_to_float(g[i])) * bf16_to_float(u[i]);
+        for (int32_t b = 0; b < nb; ++b) {
+            float amax = 0.0f;
+            for (int32_t i = 0; i < 128; ++i) {
+                float v = fabsf(a[b * 128 + i]);
+                if (v > amax)
+                    amax = v;
+            }
+            float scale = 0.0f;
+            if (amax > 0.0f)
+                scale = amax / 448.0f;
+            for (int32_t i = 0; i < 128; ++i)
+                act[r * I + b * 128 + i] =
+                    amax > 0.0f ? oracle_e4m3_from_float(a[b * 128 + i] / scale) : 0x00;
+            if (col_major)
+                act_scale[(int64_t)b * rows_cap + r] = scale;
+            else
+                act_scale[r * nb + b] = scale;
+        }
+    }
+    free(a);
+}
+
+/*
+ * Router top-k ("Lower latency and higher throughput with multi-node DeepSeek
+ * deployment", section "Roteador MoE": one top-k with index tracking serves all
+ * MoE models; plain top-k is the special case of group-limited top-k with a
+ * single group).  For each token's logits l[0..E):
+ *   - experts form n_group contiguous groups of E/n_group; a group's score is
+ *     its largest logit; the topk_group best groups are kept (ties: lower
+ *     group id);
+ *   - the k largest logits among the kept groups' experts are chosen, best
+ *     first (ties: lower expert id);
+ *   - weights: score_fn 0 = softmax: exp(l_j - m) / sum, the sum over the k
+ *     chosen (renormalize) or over all E logits; score_fn 1 = sigmoid:
+ *     s_j = 1/(1+exp(-l_j)), divided by the sum of the chosen s (renormalize)
+ *     or as is.
+ * Selection compares logits only (softmax and sigmoid are increasing), so it
+ * is exact; the weights are computed in fp64.
+ */
+void oracle_router_topk(int32_t T, int32_t E, int32_t k, const float *logits, int32_t score_fn,
+                        int32_t n_group, int32_t topk_group, int32_t renormalize,
+                        int32_t *topk_idx, float *topk_w)
+{
+    const int32_t gsize = E / n_group;
+    char *group_kept = (char *)malloc((size_t)n_group);
+    char *taken = (char *)malloc((size_t)E);
+    for (int32_t t = 0; t < T; ++t) {
+        const float *l = logits + (int64_t)t * E;
+        for (int32_t g = 0; g < n_group; ++g)
+            group_kept[g] = 0;
+        for (int32_t pick = 0; pick < topk_group; ++pick) {
+            int32_t best = -1;
+            float best_score = 0.0f;
+            for (int32_t g = 0; g < n_group; ++g) {
+                if (group_kept[g])
+                    continue;
+                float gmax = l[g * gsize];
+                for (int32_t i = 1; i < gsize; ++i)
+                    if (l[g * gsize + i] > gmax)
+                        gmax = l[g * gsize + i];
+                if (best < 0 || gmax > best_score) {
+                    best = g;
+                    best_score = gmax;
+                }
+            }
+            group_kept[best] = 1;
+        }
+        for (int32_t e = 0; e < E; ++e)
+            taken[e] = 0;
+        for (int32_t j = 0; j < k; ++j) {
+            int32_t best = -1;
+            for (int32_t e = 0; e < E; ++e) {
+                if (taken[e] || !group_kept[e / gsize])
+                    continue;
+                if (best < 0 || l[e] > l[best])
+                    best = e;
+            }
+            taken[best] = 1;
+            topk_idx[(int64_t)t * k + j] = best;
+        }
+        double w[64];
+        double sum = 0.0;
+        if (score_fn == 0) {
+            double m = l[topk_idx[(int64_t)t * k]]; /* the largest chosen logit */
+            if (!renormalize)
+                for (int32_t e = 0; e < E; ++e)
+                    if (l[e] > m)
+                        m = l[e];
+            for (int32_t j = 0; j < k; ++j)
+                w[j] = exp((double)l[topk_idx[(int64_t)t * k + j]] - m);
+            if (renormalize)
+                for (int32_t j = 0; j < k; ++j)
+                    sum += w[j];
+            else
+                for (int32_t e = 0; e < E; ++e)
+                    sum += exp((double)l[e] - m);
+            for (int32_t j = 0; j < k; ++j)
+                w[j] /= sum;
+        } else {
+            for (int32_t j = 0; j < k; ++j) {
+                w[j] = 1.0 / (1.0 + exp(-(double)l[topk_idx[(int64_t)t * k + j]]));
+                sum += w[j];
+            }
+            if (renormalize)
+                for (int32_t j = 0; j < k; ++j)
+                    w[j] /= sum;
+        }
+        for (int32_t j = 0; j < k; ++j)
+            topk_w[(int64_t)t * k + j] = (float)w[j];
+    }
+    free(group_kept);
+    free(taken);
+}

@@ -1,0 +1,152 @@
+"""GPU parity of the rows next to dispatch/combine: sender-side partial combine,
+expert-side SiLU + block-fp8 quantiser, and the router top-k.  Each is compared
+with the CPU oracle on the same seeded inputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests._lib import bf16_from_dev, bf16_to_dev, to_dev
+from workloads import (WORKLOADS, bf16_bits_to_f32, f32_to_bf16_bits, make_inputs,
+                       make_router_logits, normal_bf16_rows, random_problem)
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import combine_route_meta_b200 as moe
+
+
+def _bf16_ulp(v):
+    a = np.abs(v.astype(np.float64))
+    return np.where(a == 0, 2.0 ** -133, np.exp2(np.floor(np.log2(np.maximum(a, 1e-300))) - 7))
+
+
+# ---- sender-side (per-rank) partial combine -------------------------------------
+
+@pytest.mark.parametrize("name,E,R,H,T", [("dsv3_decode", 256, 8, 7168, None),
+                                          ("kimi_decode", 384, 16, 7168, None),
+                                          ("random", 16, 16, 1032, 300),
+                                          ("random", 64, 1, 256, 500),
+                                          ("random", 64, 4, 2048, 3000)])
+def test_rank_partial_combine(name, E, R, H, T):
+    if name == "random":
+        x, idx, w = random_problem(E + T, T, H, E, 8 if E >= 8 else 2)
+        fp8 = False
+    else:
+        wl, x, idx, w = make_inputs(name)
+        fp8 = wl.fp8
+    d = moe.dispatch(bf16_to_dev(x), to_dev(idx), to_dev(w), E, R, fp8)
+    rows = d.recv_x.shape[0]
+    eo = normal_bf16_rows(7, 3, 0, rows, H)
+    y, partial, prank, npart = moe.combine_rank_partial(d.handle, d.rank_offset, bf16_to_dev(eo))
+    assert moe.check() == 0
+    slot = d.handle.slot.cpu().numpy()
+    o = oracle.combine_rank_partial(idx, slot, w, eo, E=E, R=R)
+    np.testing.assert_array_equal(npart.cpu().numpy(), o["npart"])
+    gp = bf16_from_dev(partial)
+    n = o["npart"]
+    for t in range(idx.shape[0]):
+        np.testing.assert_array_equal(prank.cpu().numpy()[t, :n[t]], o["partial_rank"][t, :n[t]])
+        a = bf16_bits_to_f32(gp[t, :n[t]]).astype(np.float64)
+        b = bf16_bits_to_f32(o["partial"][t, :n[t]]).astype(np.float64)
+        # fp32 accumulation vs fp64 can only move a partial by one bf16 unit
+        assert np.all(np.abs(a - b) <= _bf16_ulp(b) * 1.0001), t
+    # stage 2: y is the bf16 rounding of the GPU's own partials summed in binary32, q ascending
+    acc = np.zeros((idx.shape[0], H), np.float32)
+    for q in range(idx.shape[1]):
+        m = q < n
+        acc[m] += bf16_bits_to_f32(gp[m, q])
+    want = torch.from_numpy(acc).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(bf16_from_dev(y), want)
+    # and against the oracle's y: the combine tolerance plus the partials' rounding
+    yf = bf16_bits_to_f32(bf16_from_dev(y)).astype(np.float64)
+    slack = np.abs(bf16_bits_to_f32(o["partial"]).astype(np.float64))
+    bound = 1e-2 + 4e-3 * np.abs(o["y"]) + (_bf16_ulp(bf16_bits_to_f32(o["partial"])) * (slack > 0)).sum(1)
+    assert np.all(np.abs(yf - o["y"]) <= bound)
+
+
+# ---- expert-side SiLU + block-fp8 quantiser ---------------------------------------
+
+def _silu_problem(rows, I, seed, pad_frac=0.2):
+    rng = np.random.default_rng(seed)
+    gu = f32_to_bf16_bits((rng.standard_normal((rows, 2 * I)) * 2).astype(np.float32))
+    src = np.arange(rows, dtype=np.int32)
+    src[rng.random(rows) < pad_frac] = -1
+    return gu, src
+
+
+@pytest.mark.parametrize("rows,I,in_use,col_major", [(1024, 2048, 1000, False), (1024, 2048, 1024, True),
+                                                     (300, 384, 299, False), (70, 1152, 0, False),
+                                                     (4096, 2048, 4000, True)])
+def test_silu_quant_bit_exact(rows, I, in_use, col_major):
+    gu, src = _silu_problem(rows, I, rows + I)
+    act_ref, sc_ref = oracle.silu_quant(gu, src, in_use, col_major=col_major, fill=0xA5)
+    shape = (I // 128, rows) if col_major else (rows, I // 128)
+    act = torch.full((rows, I), 0xA5, dtype=torch.uint8, device="cuda")
+    sc = torch.zeros(shape, dtype=torch.float32, device="cuda")
+    sc.view(torch.uint8).fill_(0xA5)
+    moe.silu_quant_into(bf16_to_dev(gu), to_dev(src), to_dev(np.array([in_use], np.int32)),
+                        act, sc, col_major=col_major)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(act.cpu().numpy(), act_ref)
+    np.testing.assert_array_equal(sc.cpu().numpy().view(np.uint32), sc_ref.view(np.uint32))
+
+
+def test_silu_quant_every_bf16_gate_value():
+    # gate runs through every finite bf16 value (up = 1), so the binary32 SiLU is
+    # checked against the oracle's on its whole input domain
+    bits = np.arange(0, 0x10000, dtype=np.uint32)
+    bits = bits[((bits >> 7) & 0xFF) != 0xFF].astype(np.uint16)
+    I = 2048
+    rows = (len(bits) + I - 1) // I
+    g = np.resize(bits, rows * I).reshape(rows, I)
+    gu = np.concatenate([g, np.full((rows, I), 0x3F80, np.uint16)], axis=1)
+    src = np.arange(rows, dtype=np.int32)
+    act_ref, sc_ref = oracle.silu_quant(gu, src, rows)
+    act, sc = moe.silu_quant(bf16_to_dev(gu), to_dev(src), to_dev(np.array([rows], np.int32)))
+    np.testing.assert_array_equal(act.view(torch.uint8).cpu().numpy(), act_ref)
+    np.testing.assert_array_equal(sc.cpu().numpy().view(np.uint32), sc_ref.view(np.uint32))
+
+
+def test_silu_quant_on_a_dispatch_layout():
+    # rows_in_use and padding come from a real PAD128 dispatch
+    wl, x, idx, w = make_inputs("sweep_256", H=256)
+    d = moe.dispatch(bf16_to_dev(x), to_dev(idx), to_dev(w), wl.E, wl.R, True, pad128=True)
+    rows = d.recv_x.shape[0]
+    I = 2048
+    gu, _ = _silu_problem(rows, I, 11, pad_frac=0.0)
+    act, sc = moe.silu_quant(bf16_to_dev(gu), d.recv_src, d.expert_offset[wl.E:])
+    src = d.recv_src.cpu().numpy()
+    act_ref, sc_ref = oracle.silu_quant(gu, src, int(d.expert_offset[wl.E].item()))
+    np.testing.assert_array_equal(act.view(torch.uint8).cpu().numpy(), act_ref)
+    np.testing.assert_array_equal(sc.cpu().numpy().view(np.uint32), sc_ref.view(np.uint32))
+
+
+# ---- router top-k ---------------------------------------------------------------------
+
+@pytest.mark.parametrize("T,E,k,fn,G,TG,renorm", [
+    (128, 256, 8, "sigmoid", 1, 1, True),
+    (128, 256, 8, "sigmoid", 8, 4, True),     # DeepSeek-V3-shaped group-limited routing
+    (128, 384, 8, "softmax", 1, 1, True),
+    (4096, 256, 8, "softmax", 1, 1, False),
+    (1000, 64, 6, "softmax", 8, 3, True),
+    (7, 1024, 32, "sigmoid", 32, 2, False),
+    (33, 8, 2, "softmax", 2, 2, True),
+])
+def test_router_topk(T, E, k, fn, G, TG, renorm):
+    l = np.random.default_rng(T + E).standard_normal((T, E)).astype(np.float32)
+    l[0, 3] = l[0, 5] = l[0].max() + 1.0            # a tie: the lower id comes first
+    ref_idx, ref_w = oracle.router_topk(l, k, score_fn=fn, n_group=G, topk_group=TG, renormalize=renorm)
+    idx, w = moe.router_topk(to_dev(l), k, score_fn=fn, n_group=G, topk_group=TG, renormalize=renorm)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
+    np.testing.assert_allclose(w.cpu().numpy(), ref_w, rtol=2e-6, atol=1e-9)
+
+
+@pytest.mark.parametrize("name,fn", [("tiny", "softmax"), ("dsv3_decode", "sigmoid")])
+def test_router_feeds_dispatch_like_the_generator(name, fn):
+    wl = WORKLOADS[name]
+    logits = make_router_logits(wl).astype(np.float32)
+    idx, w = moe.router_topk(to_dev(logits), wl.k, score_fn=fn)
+    ref_idx, ref_w = oracle.router_topk(logits, wl.k, score_fn=fn)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
+    np.testing.assert_allclose(w.cpu().numpy(), ref_w, rtol=2e-6)

@@ -116,6 +116,13 @@ def _topk_desc(scores: np.ndarray, k: int) -> np.ndarray:
     return np.argsort(-scores, axis=1, kind="stable")[:, :k].astype(np.int32)
 
 
+def make_router_logits(w: Workload) -> np.ndarray:
+    """The N(0,1) router logits[T,E] (float64) behind the softmax / sigmoid workloads."""
+    if w.routing not in ("softmax_topk", "sigmoid_topk"):
+        raise ValueError(f"{w.name} draws its routing without logits")
+    return _rng(w.seed, _STREAM_ROUTING).standard_normal((w.T, w.E))
+
+
 def make_routing(w: Workload) -> tuple[np.ndarray, np.ndarray]:
     """Router choices topk_idx[T,k] (int32) and weights topk_w[T,k] (float32)."""
     rng = _rng(w.seed, _STREAM_ROUTING)
