@@ -14,10 +14,11 @@
 // Softmax and sigmoid are increasing, so the choice compares logits only and
 // is exact; the weights use expf and IEEE division.
 //
-// One warp per token: the logits go to shared memory, lane g scores group g,
-// and each pick is a warp-wide argmax of (value, id) pairs (larger value, then
-// smaller id) over each lane's best remaining candidate; lane e % 32 owns
-// expert e and keeps a bitmask of its experts already taken.
+// One warp per token: the logits go to shared memory, the lanes fold them into
+// per-group maxima with shared-memory atomics, and each pick is a warp-wide
+// argmax of (value, id) pairs (larger value, then smaller id) over each lane's
+// best remaining candidate; lane e % 32 owns expert e and keeps a bitmask of
+// its experts already taken.
 #pragma once
 
 #include "common.cuh"
@@ -50,6 +51,18 @@ __device__ __forceinline__ void warp_argmax(float &v, int32_t &id)
     }
 }
 
+// A signed integer that orders like the float it comes from (finite values).
+__device__ __forceinline__ int32_t ordered_key(float f)
+{
+    const int32_t i = __float_as_int(f);
+    return i >= 0 ? i : (int32_t)(0x80000000u - (uint32_t)i);
+}
+
+__device__ __forceinline__ float key_value(int32_t k)
+{
+    return __int_as_float(k >= 0 ? k : (int32_t)(0x80000000u - (uint32_t)k));
+}
+
 __device__ __forceinline__ float warp_sum(float v)
 {
 #pragma unroll
@@ -62,9 +75,11 @@ __global__ void __launch_bounds__(kRouterWarps * kWarp) router_topk(RouterArgs a
 {
     stream_order_begin();
     __shared__ float s_l[kRouterWarps][kRouterMaxE];
+    __shared__ int32_t s_g[kRouterWarps][kRouterMaxGroups];
     const int warp = threadIdx.x / kWarp;
     const int32_t lane = (int32_t)lane_id();
     float *sl = s_l[warp];
+    int32_t *sg = s_g[warp];
     const int32_t gsize = a.E / a.n_group;
     const int32_t per_lane = (a.E + kWarp - 1) / kWarp;
     const float neg_inf = -__int_as_float(0x7f800000);
@@ -75,19 +90,24 @@ __global__ void __launch_bounds__(kRouterWarps * kWarp) router_topk(RouterArgs a
             sl[e] = __ldg(l + e);
         __syncwarp();
 
-        // groups
-        float gscore = neg_inf;
-        if (lane < a.n_group) {
-            gscore = sl[lane * gsize];
-            for (int32_t i = 1; i < gsize; ++i)
-                gscore = fmaxf(gscore, sl[lane * gsize + i]);
-        }
-        uint32_t kept = 0;
-        for (int32_t p = 0; p < a.topk_group; ++p) {
-            float v = (lane < a.n_group && !((kept >> lane) & 1u)) ? gscore : neg_inf;
-            int32_t id = lane < a.n_group ? lane : INT32_MAX;
-            warp_argmax(v, id);
-            kept |= 1u << id;
+        // groups: every lane folds its own experts into the group maxima (order-
+        // preserving integer keys, shared-memory atomics), then lane g reads group g
+        uint32_t kept = 0xffffffffu;
+        if (a.n_group > 1) {
+            if (lane < a.n_group)
+                sg[lane] = INT32_MIN;
+            __syncwarp();
+            for (int32_t e = lane; e < a.E; e += kWarp)
+                atomicMax(&sg[e / gsize], ordered_key(sl[e]));
+            __syncwarp();
+            const float gscore = lane < a.n_group ? key_value(sg[lane]) : neg_inf;
+            kept = 0;
+            for (int32_t p = 0; p < a.topk_group; ++p) {
+                float v = (lane < a.n_group && !((kept >> lane) & 1u)) ? gscore : neg_inf;
+                int32_t id = lane < a.n_group ? lane : INT32_MAX;
+                warp_argmax(v, id);
+                kept |= 1u << id;
+            }
         }
 
         // experts: lane owns e = lane + 32 i
