@@ -249,7 +249,7 @@ def graph_kernels(g):
 
 
 def short_kernel_name(mangled):
-    for k in ("dispatch_fused", "scatter_bulk_bf16", "scatter_rows", "combine_rows",
+    for k in ("dispatch_fused", "dispatch_direct", "scatter_bulk_bf16", "scatter_rows", "combine_rows",
               "meta_single_block", "meta_tile_count", "meta_tile_scan", "meta_tile_assign"):
         if k in mangled:
             return k

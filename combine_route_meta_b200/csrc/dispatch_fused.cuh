@@ -159,4 +159,153 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_fused(FusedArgs 
     }
 }
 
+// ---- direct-rank variant (no padding) -----------------------------------------
+// Without padding the stable (token, k) order gives each entry a closed-form
+// slot: for entry (t, j) with expert e,
+//   slot = #{entries with expert < e} + #{entries (t', j') before (t, j) with expert e},
+// the first term being the unpadded offset of e and the second its rank within
+// e.  A token's CTA counts both terms for its own k experts while its row is in
+// flight: each thread compares its share of the S expert ids with the k own ids,
+// the two counts of entry j travel packed in one 32-bit word (low and high
+// halves, S <= kFusedMaxEntries < 2^16), and a warp reduction plus one barrier
+// finish them, so no per-expert histogram or scan sits on the token's path.
+// One extra CTA (blockIdx.x == T) writes the per-expert counts and offsets, the
+// rank offsets and the unused rows' recv_src, and flags bad expert ids.
+template <int kChunks, bool kFp8, int kK>
+__global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct(FusedArgs a)
+{
+    stream_order_begin();
+    extern __shared__ int32_t sm[];
+    __shared__ uint32_t s_part[kFusedMaxThreads / kWarp][kK];
+    __shared__ int32_t s_slot[kK];
+    __shared__ int32_t s_own[kK];
+
+    const int32_t t = blockIdx.x;
+    const int nt = blockDim.x;
+    const int nwarps = nt / kWarp;
+    const int warp = threadIdx.x / kWarp;
+    const unsigned lane = lane_id();
+    const int64_t S = (int64_t)a.T * a.k;
+
+    if (t == a.T) {
+        // metadata CTA: histogram, scan, offsets, unused rows
+        int32_t *hist = sm, *off = sm + a.E;
+        for (int32_t e = threadIdx.x; e < a.E; e += nt)
+            hist[e] = 0;
+        __syncthreads();
+        for (int64_t base = 0; base < S; base += (int64_t)nt * kFusedLoadRounds) {
+            int32_t ev[kFusedLoadRounds];
+#pragma unroll
+            for (int r = 0; r < kFusedLoadRounds; ++r) {
+                const int64_t i = base + (int64_t)r * nt + threadIdx.x;
+                ev[r] = i < S ? __ldg(a.topk_idx + i) : -1;
+            }
+#pragma unroll
+            for (int r = 0; r < kFusedLoadRounds; ++r) {
+                const int64_t i = base + (int64_t)r * nt + threadIdx.x;
+                const int32_t e = ev[r];
+                if (i < S && (e < 0 || e >= a.E))
+                    raise_error(a.err, MOE_DEV_BAD_INDEX);
+                else if (i < S)
+                    atomicAdd(&hist[e], 1);
+            }
+        }
+        __syncthreads();
+        block_offsets(hist, off, a.E, 0);
+        for (int32_t e = threadIdx.x; e < a.E; e += nt) {
+            a.expert_count[e] = hist[e];
+            a.expert_offset[e] = off[e];
+        }
+        if (threadIdx.x == 0)
+            a.expert_offset[a.E] = off[a.E];
+        for (int32_t r = threadIdx.x; r <= a.R; r += nt)
+            a.rank_offset[r] = off[(int64_t)r * (a.E / a.R)];
+        block_fill_unused(a.rows_cap, a.E, a.recv_src, hist, off, 0, 1);
+        return;
+    }
+
+    constexpr int L = kFusedLaneCols;
+    const int32_t chunks = (a.H + chunk_cols<L>() - 1) / chunk_cols<L>();
+
+    // 1. The row's loads go out first: warp w owns chunks w, w + nwarps, ...
+    const uint16_t *xr = a.x + (int64_t)t * a.H;
+    LaneData<L> d[kChunks];
+#pragma unroll
+    for (int i = 0; i < kChunks; ++i) {
+        const int32_t c = warp + i * nwarps;
+        if (c < chunks)
+            load_chunk<L, kFp8>(xr, a.H, c, d[i]);
+    }
+
+    // 2. Own expert ids (broadcast loads) and this thread's share of all ids.
+    const int64_t mine = (int64_t)t * a.k;
+    constexpr int32_t kNone = 0x7fffffff; // never below or equal to a valid id
+    int32_t own[kK];
+#pragma unroll
+    for (int j = 0; j < kK; ++j) {
+        int32_t e = j < a.k ? __ldg(a.topk_idx + mine + j) : -1;
+        own[j] = (e >= 0 && e < a.E) ? e : -1;
+    }
+    if ((int)threadIdx.x < a.k) {
+        const int32_t e = __ldg(a.topk_idx + mine + threadIdx.x);
+        s_own[threadIdx.x] = (e >= 0 && e < a.E) ? e : -1;
+    }
+    uint32_t cnt[kK];
+#pragma unroll
+    for (int j = 0; j < kK; ++j)
+        cnt[j] = 0;
+    for (int64_t base = 0; base < S; base += (int64_t)nt * kFusedLoadRounds) {
+        int32_t ev[kFusedLoadRounds];
+#pragma unroll
+        for (int r = 0; r < kFusedLoadRounds; ++r) {
+            const int64_t i = base + (int64_t)r * nt + threadIdx.x;
+            ev[r] = i < S ? __ldg(a.topk_idx + i) : kNone;
+        }
+#pragma unroll
+        for (int r = 0; r < kFusedLoadRounds; ++r) {
+            const int64_t i = base + (int64_t)r * nt + threadIdx.x;
+            const int32_t e = (ev[r] >= 0 && ev[r] < a.E) ? ev[r] : kNone;
+#pragma unroll
+            for (int j = 0; j < kK; ++j)
+                cnt[j] += (uint32_t)(e < own[j]) + ((uint32_t)(e == own[j] && i < mine + j) << 16);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < kK; ++j) {
+        const uint32_t w = __reduce_add_sync(kFullMask, cnt[j]);
+        if (lane == 0)
+            s_part[warp][j] = w;
+    }
+    __syncthreads();
+
+    // 3. This token's slots: warp j adds the per-warp counts of entry j.
+    for (int j = warp; j < a.k; j += nwarps) {
+        const uint32_t v = (int)lane < nwarps ? s_part[lane][j] : 0u;
+        const uint32_t tot = __reduce_add_sync(kFullMask, v);
+        if (lane == 0) {
+            int32_t s = -1;
+            if (s_own[j] >= 0) {
+                const int64_t row = (int64_t)(tot & 0xffffu) + (tot >> 16);
+                if (row < a.rows_cap) {
+                    s = (int32_t)row;
+                    a.recv_src[row] = (int32_t)(mine + j);
+                } else {
+                    raise_error(a.err, MOE_DEV_CAPACITY);
+                }
+            }
+            a.slot[mine + j] = s;
+            s_slot[j] = s;
+        }
+    }
+    __syncthreads();
+
+    // 4. Payload to the k slots.
+#pragma unroll
+    for (int i = 0; i < kChunks; ++i) {
+        const int32_t c = warp + i * nwarps;
+        if (c < chunks)
+            store_chunk<L, kFp8>(a.recv_x, a.recv_scale, a.H, c, a.k, s_slot, a.rows_cap, a.err, d[i]);
+    }
+}
+
 } // namespace moe

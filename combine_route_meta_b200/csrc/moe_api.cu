@@ -179,6 +179,37 @@ cudaError_t launch_fused(int per, unsigned grid, unsigned block, size_t smem, cu
     }
 }
 
+template <bool kFp8, int kK>
+cudaError_t launch_direct_k(int per, unsigned grid, unsigned block, size_t smem, cudaStream_t s,
+                            const FusedArgs &f)
+{
+    switch (per) {
+    case 1:
+        return launch(dispatch_direct<1, kFp8, kK>, grid, block, smem, s, f);
+    case 2:
+        return launch(dispatch_direct<2, kFp8, kK>, grid, block, smem, s, f);
+    default:
+        return launch(dispatch_direct<4, kFp8, kK>, grid, block, smem, s, f);
+    }
+}
+
+// The fused dispatch of one token per CTA: the direct-rank form without
+// padding (T token CTAs and one metadata CTA), the histogram form with it.
+cudaError_t launch_small(bool fp8, int per, int32_t T, unsigned block, cudaStream_t s,
+                         const FusedArgs &f)
+{
+    const size_t smem = fused_smem(f.E);
+    if (f.pad128)
+        return fp8 ? launch_fused<true>(per, T, block, smem, s, f)
+                   : launch_fused<false>(per, T, block, smem, s, f);
+    const unsigned grid = (unsigned)T + 1;
+    if (f.k <= 8)
+        return fp8 ? launch_direct_k<true, 8>(per, grid, block, smem, s, f)
+                   : launch_direct_k<false, 8>(per, grid, block, smem, s, f);
+    return fp8 ? launch_direct_k<true, kFusedMaxK>(per, grid, block, smem, s, f)
+               : launch_direct_k<false, kFusedMaxK>(per, grid, block, smem, s, f);
+}
+
 size_t workspace_bytes(const moe_config *c, int32_t T)
 {
     const int64_t S = (int64_t)T * c->k;
@@ -416,9 +447,7 @@ int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
         f.recv_src = out->recv_src;
         f.slot = slot;
         f.err = dev_err;
-        const cudaError_t e =
-            fp8 ? launch_fused<true>(per, T, fused_block, fused_smem(cfg->E), s, f)
-                : launch_fused<false>(per, T, fused_block, fused_smem(cfg->E), s, f);
+        const cudaError_t e = launch_small(fp8, per, T, fused_block, s, f);
         if ((st = launched(e)) != MOE_OK)
             return st;
     } else {
