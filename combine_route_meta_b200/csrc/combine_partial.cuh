@@ -18,7 +18,8 @@
 // [rank_offset[r], rank_offset[r+1])), so the handle needs no expert ids.
 // Layout: partial [T, k, H] bf16 (rows q >= npart[t] untouched),
 // partial_rank [T, k], npart [T].  Both stages are one CTA per (token, part)
-// with one 16-byte vector per thread, like combine_rows.
+// with one 16-byte vector per thread, like combine_rows; the send stage works
+// out the token's partials afresh in every unit (a warp-wide step for k <= 32).
 #pragma once
 
 #include "common.cuh"
@@ -76,11 +77,90 @@ __device__ __forceinline__ uint4 pack_row(const float (&acc)[8])
                       pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
 }
 
+// Entry j's slot, and the partial it belongs to (-1 if dropped), into shared
+// memory; *n = the token's number of partials.  Part 0 also writes the token's
+// partial ranks and count.  For k <= 32, warp 0 does it with one lane per entry:
+// lanes holding the same rank find each other (match_any), the first of them
+// opens a partial, and an entry's partial is the number of partials opened
+// before its rank's first entry.  Larger k takes one thread, in order.
+__device__ __forceinline__ void partial_layout(const PartialArgs &a, int32_t t, int32_t part,
+                                               int32_t *s_slot, int32_t *s_q, int32_t *s_rank,
+                                               int32_t *n_out)
+{
+    const int64_t base = (int64_t)t * a.k;
+    if (a.k <= kWarp) {
+        if (threadIdx.x >= kWarp)
+            return;
+        const int32_t j = (int32_t)lane_id();
+        int32_t s = -1, r = -1 - j; // dropped entries get ranks nobody shares
+        bool valid = false;
+        if (j < a.k) {
+            s = __ldg(a.slot + base + j);
+            if (s >= 0 && s < a.rows_cap) {
+                valid = true;
+                r = rank_of_row(a.rank_offset, a.R, s);
+            } else {
+                if (s != -1)
+                    raise_error(a.err, MOE_DEV_BAD_SLOT);
+                s = -1;
+            }
+        }
+        const unsigned same = __match_any_sync(kFullMask, r);
+        const int32_t first = __ffs(same) - 1;
+        const unsigned opens = __ballot_sync(kFullMask, valid && first == j);
+        const int32_t q = valid ? __popc(opens & ((1u << first) - 1u)) : -1;
+        if (j < a.k) {
+            s_slot[j] = s;
+            s_q[j] = q;
+        }
+        if (part == 0 && valid && first == j)
+            a.partial_rank[base + q] = r;
+        if (j == 0) {
+            *n_out = __popc(opens);
+            if (part == 0)
+                a.npart[t] = __popc(opens);
+        }
+        return;
+    }
+    if (threadIdx.x != 0)
+        return;
+    int32_t n = 0;
+    for (int32_t j = 0; j < a.k; ++j) {
+        int32_t s = __ldg(a.slot + base + j);
+        if (!(s >= 0 && s < a.rows_cap)) {
+            if (s != -1)
+                raise_error(a.err, MOE_DEV_BAD_SLOT);
+            s_slot[j] = -1;
+            s_q[j] = -1;
+            continue;
+        }
+        const int32_t r = rank_of_row(a.rank_offset, a.R, s);
+        int32_t q = 0;
+        while (q < n && s_rank[q] != r)
+            ++q;
+        if (q == n) {
+            s_rank[n++] = r;
+            if (part == 0)
+                a.partial_rank[base + q] = r;
+        }
+        s_slot[j] = s;
+        s_q[j] = q;
+    }
+    *n_out = n;
+    if (part == 0)
+        a.npart[t] = n;
+}
+
+// kAllRows (k <= kCombineBatch): every receive row of the token is loaded at
+// once, then the partials are formed from registers one after another.
+// Otherwise each partial loads its own rows, kCombineBatch at a time.
+template <bool kAllRows>
 __global__ void __launch_bounds__(kPartialThreads) combine_partial_send(PartialArgs a)
 {
     stream_order_begin();
     __shared__ int32_t s_slot[kPartialMaxK];
     __shared__ int32_t s_q[kPartialMaxK]; // partial index of entry j, -1 if dropped
+    __shared__ int32_t s_rank[kPartialMaxK];
     __shared__ int32_t s_n;
     const int32_t nvec = a.H / 8;
     const int64_t units = (int64_t)a.T * a.parts;
@@ -88,61 +168,60 @@ __global__ void __launch_bounds__(kPartialThreads) combine_partial_send(PartialA
         const int32_t t = (int32_t)(u / a.parts);
         const int32_t part = (int32_t)(u % a.parts);
         __syncthreads(); // the previous unit is done with the shared arrays
-        if (threadIdx.x == 0) {
-            // slots, their ranks, and each entry's partial (distinct ranks in order)
-            int32_t ranks[kPartialMaxK];
-            int32_t n = 0;
-            for (int32_t j = 0; j < a.k; ++j) {
-                int32_t s = __ldg(a.slot + (int64_t)t * a.k + j);
-                if (!(s >= 0 && s < a.rows_cap)) {
-                    if (s != -1)
-                        raise_error(a.err, MOE_DEV_BAD_SLOT);
-                    s_slot[j] = -1;
-                    s_q[j] = -1;
-                    continue;
-                }
-                const int32_t r = rank_of_row(a.rank_offset, a.R, s);
-                int32_t q = 0;
-                while (q < n && ranks[q] != r)
-                    ++q;
-                if (q == n) {
-                    ranks[n++] = r;
-                    if (part == 0)
-                        a.partial_rank[(int64_t)t * a.k + q] = r;
-                }
-                s_slot[j] = s;
-                s_q[j] = q;
-            }
-            s_n = n;
-            if (part == 0)
-                a.npart[t] = n;
-        }
+        partial_layout(a, t, part, s_slot, s_q, s_rank, &s_n);
         __syncthreads();
         const int32_t v = part * kPartialThreads + (int32_t)threadIdx.x;
         if (v >= nvec)
             continue;
         const int32_t n = s_n;
-        for (int32_t q = 0; q < n; ++q) {
-            float acc[8];
+        const float *ws = a.w + (int64_t)t * a.k;
+        uint16_t *out = a.partial + (int64_t)t * a.k * a.H + (int64_t)v * 8;
+        if constexpr (kAllRows) {
+            uint4 r[kCombineBatch];
+            float wv[kCombineBatch];
+            int32_t qv[kCombineBatch];
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                acc[i] = 0.0f;
-            for (int32_t j0 = 0; j0 < a.k; j0 += kCombineBatch) {
-                uint4 r[kCombineBatch];
-                bool use[kCombineBatch];
-#pragma unroll
-                for (int jj = 0; jj < kCombineBatch; ++jj) {
-                    const int32_t j = j0 + jj;
-                    use[jj] = j < a.k && s_q[j] == q;
-                    r[jj] = use[jj] ? ld_stream_v4(a.expert_out + (int64_t)s_slot[j] * a.H + (int64_t)v * 8)
-                                    : make_uint4(0u, 0u, 0u, 0u);
-                }
-#pragma unroll
-                for (int jj = 0; jj < kCombineBatch; ++jj)
-                    if (use[jj])
-                        fma_row(acc, __ldg(a.w + (int64_t)t * a.k + j0 + jj), r[jj]);
+            for (int j = 0; j < kCombineBatch; ++j) {
+                const bool use = j < a.k && s_q[j] >= 0;
+                qv[j] = use ? s_q[j] : -1;
+                r[j] = use ? ld_stream_v4(a.expert_out + (int64_t)s_slot[j] * a.H + (int64_t)v * 8)
+                           : make_uint4(0u, 0u, 0u, 0u);
+                wv[j] = use ? __ldg(ws + j) : 0.0f;
             }
-            st_v4(a.partial + ((int64_t)t * a.k + q) * a.H + (int64_t)v * 8, pack_row(acc));
+            for (int32_t q = 0; q < n; ++q) {
+                float acc[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    acc[i] = 0.0f;
+#pragma unroll
+                for (int j = 0; j < kCombineBatch; ++j)
+                    if (qv[j] == q)
+                        fma_row(acc, wv[j], r[j]);
+                st_v4(out + (int64_t)q * a.H, pack_row(acc));
+            }
+        } else {
+            for (int32_t q = 0; q < n; ++q) {
+                float acc[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    acc[i] = 0.0f;
+                for (int32_t j0 = 0; j0 < a.k; j0 += kCombineBatch) {
+                    uint4 r[kCombineBatch];
+                    bool use[kCombineBatch];
+#pragma unroll
+                    for (int jj = 0; jj < kCombineBatch; ++jj) {
+                        const int32_t j = j0 + jj;
+                        use[jj] = j < a.k && s_q[j] == q;
+                        r[jj] = use[jj] ? ld_stream_v4(a.expert_out + (int64_t)s_slot[j] * a.H + (int64_t)v * 8)
+                                        : make_uint4(0u, 0u, 0u, 0u);
+                    }
+#pragma unroll
+                    for (int jj = 0; jj < kCombineBatch; ++jj)
+                        if (use[jj])
+                            fma_row(acc, __ldg(ws + j0 + jj), r[jj]);
+                }
+                st_v4(out + (int64_t)q * a.H, pack_row(acc));
+            }
         }
     }
 }

@@ -50,7 +50,21 @@ constexpr int kVersion = 100; // 0.1.0
 struct DeviceInfo {
     bool ready = false;
     int sms = 0;
+    // resident CTAs per SM of the kernels whose grid is one wave
+    int silu_per_sm = 1;
+    int router_per_sm[4] = {1, 1, 1, 1}; // 4, 8, 16, 32 logits per lane
+    int send_per_sm[2] = {1, 1};         // combine_partial_send<false>, <true>
+    int recv_per_sm = 1;
 };
+
+template <typename K>
+int resident_per_sm(K kernel, int block, size_t smem)
+{
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, block, smem) != cudaSuccess)
+        return 0;
+    return n > 0 ? n : 1;
+}
 DeviceInfo g_dev[kMaxDevices];
 
 int device_info(DeviceInfo **out)
@@ -69,6 +83,16 @@ int device_info(DeviceInfo **out)
                                  (int)meta_assign_smem(MOE_MAX_EXPERTS)) != cudaSuccess ||
             cudaFuncSetAttribute(scatter_bulk_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kBulkMaxSmem) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        const int rb = kRouterWarps * kWarp;
+        if (!(d.silu_per_sm = resident_per_sm(silu_quant_rows, kSiluThreads, 0)) ||
+            !(d.router_per_sm[0] = resident_per_sm(router_topk<4>, rb, 0)) ||
+            !(d.router_per_sm[1] = resident_per_sm(router_topk<8>, rb, 0)) ||
+            !(d.router_per_sm[2] = resident_per_sm(router_topk<16>, rb, 0)) ||
+            !(d.router_per_sm[3] = resident_per_sm(router_topk<kRouterMaxE / kWarp>, rb, 0)) ||
+            !(d.send_per_sm[0] = resident_per_sm(combine_partial_send<false>, kPartialThreads, 0)) ||
+            !(d.send_per_sm[1] = resident_per_sm(combine_partial_send<true>, kPartialThreads, 0)) ||
+            !(d.recv_per_sm = resident_per_sm(combine_partial_recv, kPartialThreads, 0)))
             return MOE_ERR_CUDA;
         d.ready = true;
     }
@@ -603,10 +627,17 @@ int moe_combine_rank_partial(const moe_handle *handle, const int32_t *rank_offse
     a.y = static_cast<uint16_t *>(y);
     a.err = dev_err;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const unsigned grid = grid_for((int64_t)a.T * a.parts, dev->sms, 16);
-    if ((st = launched(launch(combine_partial_send, grid, kPartialThreads, 0, s, a))) != MOE_OK)
+    // one resident wave of CTAs each
+    const int64_t units = (int64_t)a.T * a.parts;
+    const bool all_rows = a.k <= kCombineBatch;
+    const unsigned send_grid = grid_for(units, dev->sms, dev->send_per_sm[all_rows ? 1 : 0]);
+    const cudaError_t e = all_rows
+                              ? launch(combine_partial_send<true>, send_grid, kPartialThreads, 0, s, a)
+                              : launch(combine_partial_send<false>, send_grid, kPartialThreads, 0, s, a);
+    if ((st = launched(e)) != MOE_OK)
         return st;
-    return launched(launch(combine_partial_recv, grid, kPartialThreads, 0, s, a));
+    return launched(launch(combine_partial_recv, grid_for(units, dev->sms, dev->recv_per_sm),
+                           kPartialThreads, 0, s, a));
 }
 
 int moe_silu_quant(int64_t rows_cap, int32_t I, const void *gate_up, const int32_t *recv_src,
@@ -638,7 +669,7 @@ int moe_silu_quant(int64_t rows_cap, int32_t I, const void *gate_up, const int32
     a.scale = act_scale;
     a.col_major = scale_col_major ? 1 : 0;
     // A fixed grid, whatever the routing: the kernel reads how many rows are in use.
-    const unsigned grid = (unsigned)(dev->sms * kSiluCtasPerSm);
+    const unsigned grid = (unsigned)(dev->sms * dev->silu_per_sm);
     return launched(launch(silu_quant_rows, grid, kSiluThreads, 0, static_cast<cudaStream_t>(stream), a));
 }
 
@@ -672,8 +703,21 @@ int moe_router_topk(int32_t T, int32_t E, int32_t k, const float *logits, int32_
     a.renormalize = renormalize ? 1 : 0;
     a.topk_idx = topk_idx;
     a.topk_w = topk_w;
-    const unsigned grid = grid_for((T + kRouterWarps - 1) / kRouterWarps, dev->sms, 16);
-    return launched(launch(router_topk, grid, kRouterWarps * kWarp, 0, static_cast<cudaStream_t>(stream), a));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const unsigned block = kRouterWarps * kWarp;
+    const int64_t units = (T + kRouterWarps - 1) / kRouterWarps;
+    // logits per lane, rounded up to a power of two; at most one wave of CTAs
+    if (E <= 4 * kWarp)
+        return launched(launch(router_topk<4>, grid_for(units, dev->sms, dev->router_per_sm[0]),
+                               block, 0, s, a));
+    if (E <= 8 * kWarp)
+        return launched(launch(router_topk<8>, grid_for(units, dev->sms, dev->router_per_sm[1]),
+                               block, 0, s, a));
+    if (E <= 16 * kWarp)
+        return launched(launch(router_topk<16>, grid_for(units, dev->sms, dev->router_per_sm[2]),
+                               block, 0, s, a));
+    return launched(launch(router_topk<kRouterMaxE / kWarp>,
+                           grid_for(units, dev->sms, dev->router_per_sm[3]), block, 0, s, a));
 }
 
 int moe_check(int32_t *dev_err, void *stream, int32_t *bits_out)

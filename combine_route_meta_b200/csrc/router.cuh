@@ -14,11 +14,13 @@
 // Softmax and sigmoid are increasing, so the choice compares logits only and
 // is exact; the weights use expf and IEEE division.
 //
-// One warp per token: the logits go to shared memory, the lanes fold them into
-// per-group maxima with shared-memory atomics, and each pick is a warp-wide
-// argmax of (value, id) pairs (larger value, then smaller id) over each lane's
-// best remaining candidate; lane e % 32 owns expert e and keeps a bitmask of
-// its experts already taken.
+// One warp per token.  Lane e % 32 keeps the logits of experts e = lane + 32 i
+// in registers, as integers that order like the floats (finite or infinite
+// logits), so every comparison is an integer one.  A pick is two warp
+// reductions (redux.sync): the largest key among the lanes' best remaining
+// candidates, then the smallest expert id holding that key.  Group maxima are
+// folded with shared-memory atomics; the topk_group picks over them use the
+// same two reductions.
 #pragma once
 
 #include "common.cuh"
@@ -28,7 +30,8 @@ namespace moe {
 constexpr int kRouterMaxE = 1024;
 constexpr int kRouterMaxK = 32;
 constexpr int kRouterMaxGroups = 32;
-constexpr int kRouterWarps = 4;
+constexpr int kRouterWarps = 8;
+constexpr int32_t kNoKey = INT32_MIN; // below every logit's key
 
 struct RouterArgs {
     const float *logits; // [T, E]
@@ -37,21 +40,7 @@ struct RouterArgs {
     float *topk_w;     // [T, k]
 };
 
-// Warp-wide best (value, id): larger value wins, equal values go to the smaller id.
-__device__ __forceinline__ void warp_argmax(float &v, int32_t &id)
-{
-#pragma unroll
-    for (int d = 16; d >= 1; d >>= 1) {
-        const float ov = __shfl_xor_sync(kFullMask, v, d);
-        const int32_t oid = __shfl_xor_sync(kFullMask, id, d);
-        if (ov > v || (ov == v && oid < id)) {
-            v = ov;
-            id = oid;
-        }
-    }
-}
-
-// A signed integer that orders like the float it comes from (finite values).
+// A signed integer that orders like the float it comes from (not NaN).
 __device__ __forceinline__ int32_t ordered_key(float f)
 {
     const int32_t i = __float_as_int(f);
@@ -71,68 +60,86 @@ __device__ __forceinline__ float warp_sum(float v)
     return v;
 }
 
+// The warp's best (key, id): largest key, then smallest id.  Lanes without a
+// candidate pass kNoKey.
+__device__ __forceinline__ int32_t warp_pick(int32_t key, int32_t id, int32_t &best_key)
+{
+    best_key = __reduce_max_sync(kFullMask, key);
+    return __reduce_min_sync(kFullMask, key == best_key ? id : INT32_MAX);
+}
+
+template <int kPer>
 __global__ void __launch_bounds__(kRouterWarps * kWarp) router_topk(RouterArgs a)
 {
     stream_order_begin();
-    __shared__ float s_l[kRouterWarps][kRouterMaxE];
     __shared__ int32_t s_g[kRouterWarps][kRouterMaxGroups];
     const int warp = threadIdx.x / kWarp;
     const int32_t lane = (int32_t)lane_id();
-    float *sl = s_l[warp];
     int32_t *sg = s_g[warp];
     const int32_t gsize = a.E / a.n_group;
-    const int32_t per_lane = (a.E + kWarp - 1) / kWarp;
     const float neg_inf = -__int_as_float(0x7f800000);
     const int64_t nwarps = (int64_t)gridDim.x * kRouterWarps;
     for (int64_t t = (int64_t)blockIdx.x * kRouterWarps + warp; t < a.T; t += nwarps) {
         const float *l = a.logits + t * a.E;
-        for (int32_t e = lane; e < a.E; e += kWarp)
-            sl[e] = __ldg(l + e);
-        __syncwarp();
-
-        // groups: every lane folds its own experts into the group maxima (order-
-        // preserving integer keys, shared-memory atomics), then lane g reads group g
-        uint32_t kept = 0xffffffffu;
-        if (a.n_group > 1) {
-            if (lane < a.n_group)
-                sg[lane] = INT32_MIN;
-            __syncwarp();
-            for (int32_t e = lane; e < a.E; e += kWarp)
-                atomicMax(&sg[e / gsize], ordered_key(sl[e]));
-            __syncwarp();
-            const float gscore = lane < a.n_group ? key_value(sg[lane]) : neg_inf;
-            kept = 0;
-            for (int32_t p = 0; p < a.topk_group; ++p) {
-                float v = (lane < a.n_group && !((kept >> lane) & 1u)) ? gscore : neg_inf;
-                int32_t id = lane < a.n_group ? lane : INT32_MAX;
-                warp_argmax(v, id);
-                kept |= 1u << id;
-            }
+        float lv[kPer];
+        int32_t key[kPer];
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int32_t e = lane + kWarp * i;
+            lv[i] = e < a.E ? __ldg(l + e) : neg_inf;
+            key[i] = e < a.E ? ordered_key(lv[i]) : kNoKey;
         }
 
-        // experts: lane owns e = lane + 32 i
-        uint32_t taken = 0;
-        int32_t my_idx = -1;  // lane j < k ends holding the j-th pick
-        float my_logit = 0.0f;
-        for (int32_t j = 0; j < a.k; ++j) {
-            float v = neg_inf;
-            int32_t id = INT32_MAX;
-            for (int32_t i = 0; i < per_lane; ++i) {
+        // groups: drop the experts of the groups that are not kept
+        if (a.n_group > 1) {
+            if (lane < a.n_group)
+                sg[lane] = kNoKey;
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < kPer; ++i) {
                 const int32_t e = lane + kWarp * i;
-                if (e >= a.E || ((taken >> i) & 1u) || !((kept >> (e / gsize)) & 1u))
-                    continue;
-                const float le = sl[e];
-                if (le > v) { // e increases with i, so ties keep the smaller id
-                    v = le;
-                    id = e;
+                if (e < a.E)
+                    atomicMax(&sg[e / gsize], key[i]);
+            }
+            __syncwarp();
+            const int32_t gkey = lane < a.n_group ? sg[lane] : kNoKey;
+            uint32_t kept = 0;
+            for (int32_t p = 0; p < a.topk_group; ++p) {
+                int32_t best;
+                const int32_t g = warp_pick((kept >> lane) & 1u ? kNoKey : gkey,
+                                            lane < a.n_group ? lane : INT32_MAX, best);
+                kept |= 1u << g;
+            }
+#pragma unroll
+            for (int i = 0; i < kPer; ++i) {
+                const int32_t e = lane + kWarp * i;
+                if (e < a.E && !((kept >> (e / gsize)) & 1u))
+                    key[i] = kNoKey;
+            }
+            __syncwarp(); // sg is rewritten by the next token
+        }
+
+        // experts: each pick marks the chosen expert taken in its lane
+        int32_t my_idx = -1; // lane j < k ends holding the j-th pick
+        float my_logit = 0.0f;
+        uint32_t taken = 0;  // bit i: expert lane + 32 i already chosen
+        for (int32_t j = 0; j < a.k; ++j) {
+            int32_t cand = kNoKey, ci = 0;
+#pragma unroll
+            for (int i = 0; i < kPer; ++i) {
+                const int32_t ki = (taken >> i) & 1u ? kNoKey : key[i];
+                if (ki > cand) { // i ascending: ties keep the smaller id
+                    cand = ki;
+                    ci = i;
                 }
             }
-            warp_argmax(v, id);
-            if (id != INT32_MAX && id % kWarp == lane)
+            int32_t best;
+            const int32_t id = warp_pick(cand, cand == kNoKey ? INT32_MAX : lane + kWarp * ci, best);
+            if (id % kWarp == lane)
                 taken |= 1u << (id / kWarp);
             if (lane == j) {
                 my_idx = id;
-                my_logit = v;
+                my_logit = key_value(best);
             }
         }
 
@@ -145,16 +152,17 @@ __global__ void __launch_bounds__(kRouterWarps * kWarp) router_topk(RouterArgs a
                 wj = lane < a.k ? expf(my_logit - m) : 0.0f;
                 denom = warp_sum(wj);
             } else {
-                float mm = neg_inf;
-                for (int32_t e = lane; e < a.E; e += kWarp)
-                    mm = fmaxf(mm, sl[e]);
+                int32_t mk = kNoKey;
 #pragma unroll
-                for (int d = 16; d >= 1; d >>= 1)
-                    mm = fmaxf(mm, __shfl_xor_sync(kFullMask, mm, d));
-                m = mm;
+                for (int i = 0; i < kPer; ++i)
+                    if (lane + kWarp * i < a.E)
+                        mk = max(mk, ordered_key(lv[i]));
+                m = key_value(__reduce_max_sync(kFullMask, mk));
                 float part = 0.0f;
-                for (int32_t e = lane; e < a.E; e += kWarp)
-                    part += expf(sl[e] - m);
+#pragma unroll
+                for (int i = 0; i < kPer; ++i)
+                    if (lane + kWarp * i < a.E)
+                        part += expf(lv[i] - m);
                 denom = warp_sum(part);
                 wj = lane < a.k ? expf(my_logit - m) : 0.0f;
             }
@@ -168,7 +176,6 @@ __global__ void __launch_bounds__(kRouterWarps * kWarp) router_topk(RouterArgs a
             a.topk_idx[t * a.k + lane] = my_idx;
             a.topk_w[t * a.k + lane] = wj;
         }
-        __syncwarp(); // the next token may overwrite the logits
     }
 }
 

@@ -23,14 +23,16 @@ def _bf16_ulp(v):
 
 # ---- sender-side (per-rank) partial combine -------------------------------------
 
-@pytest.mark.parametrize("name,E,R,H,T", [("dsv3_decode", 256, 8, 7168, None),
-                                          ("kimi_decode", 384, 16, 7168, None),
-                                          ("random", 16, 16, 1032, 300),
-                                          ("random", 64, 1, 256, 500),
-                                          ("random", 64, 4, 2048, 3000)])
-def test_rank_partial_combine(name, E, R, H, T):
+@pytest.mark.parametrize("name,E,R,H,T,k", [("dsv3_decode", 256, 8, 7168, None, 8),
+                                            ("kimi_decode", 384, 16, 7168, None, 8),
+                                            ("random", 16, 16, 1032, 300, 8),
+                                            ("random", 64, 1, 256, 500, 8),
+                                            ("random", 64, 4, 2048, 3000, 8),
+                                            ("random", 64, 8, 512, 200, 12),   # rows loaded per partial
+                                            ("random", 128, 16, 256, 100, 40)])  # layout by one thread
+def test_rank_partial_combine(name, E, R, H, T, k):
     if name == "random":
-        x, idx, w = random_problem(E + T, T, H, E, 8 if E >= 8 else 2)
+        x, idx, w = random_problem(E + T, T, H, E, k)
         fp8 = False
     else:
         wl, x, idx, w = make_inputs(name)
@@ -142,6 +144,7 @@ def test_silu_quant_on_a_dispatch_layout():
     (1000, 64, 6, "softmax", 8, 3, True),
     (7, 1024, 32, "sigmoid", 32, 2, False),
     (33, 8, 2, "softmax", 2, 2, True),
+    (300, 200, 8, "softmax", 8, 3, True),     # 25-expert groups straddle the lanes
 ])
 def test_router_topk(T, E, k, fn, G, TG, renorm):
     l = np.random.default_rng(T + E).standard_normal((T, E)).astype(np.float32)
@@ -160,3 +163,19 @@ def test_router_feeds_dispatch_like_the_generator(name, fn):
     ref_idx, ref_w = oracle.router_topk(logits, wl.k, score_fn=fn)
     np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
     np.testing.assert_allclose(w.cpu().numpy(), ref_w, rtol=2e-6)
+
+
+@pytest.mark.parametrize("E,G,TG,fn", [(256, 1, 1, "softmax"), (256, 8, 4, "sigmoid"), (96, 4, 2, "softmax"),
+                                       (384, 1, 1, "sigmoid")])
+def test_router_topk_ties_zeros_and_infinities(E, G, TG, fn):
+    # few distinct logits, so most picks are decided by the lower-id rule; signed
+    # zeros compare equal; -inf logits are the last choice
+    rng = np.random.default_rng(E + G)
+    T, k = 512, 8
+    l = (rng.integers(-3, 4, size=(T, E)) * 0.5).astype(np.float32)
+    l[rng.random((T, E)) < 0.3] = -0.0
+    l[rng.random((T, E)) < 0.1] = -np.inf
+    ref_idx, ref_w = oracle.router_topk(l, k, score_fn=fn, n_group=G, topk_group=TG, renormalize=True)
+    idx, w = moe.router_topk(to_dev(l), k, score_fn=fn, n_group=G, topk_group=TG, renormalize=True)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
+    np.testing.assert_allclose(w.cpu().numpy(), ref_w, rtol=2e-6, atol=1e-9)
