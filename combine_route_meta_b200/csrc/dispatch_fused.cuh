@@ -240,34 +240,50 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct(FusedArgs
     // 2. Own expert ids (broadcast loads) and this thread's share of all ids.
     const int64_t mine = (int64_t)t * a.k;
     constexpr int32_t kNone = 0x7fffffff; // never below or equal to a valid id
-    int32_t own[kK];
+    // Up to 8 own ids stay in registers; more are read from shared memory (the
+    // registers are needed for the row).
+    constexpr bool kOwnInRegs = kK <= 8;
+    int32_t own[kOwnInRegs ? kK : 1];
+    if constexpr (kOwnInRegs) {
 #pragma unroll
-    for (int j = 0; j < kK; ++j) {
-        int32_t e = j < a.k ? __ldg(a.topk_idx + mine + j) : -1;
-        own[j] = (e >= 0 && e < a.E) ? e : -1;
+        for (int j = 0; j < kK; ++j) {
+            const int32_t e = j < a.k ? __ldg(a.topk_idx + mine + j) : -1;
+            own[j] = (e >= 0 && e < a.E) ? e : -1;
+        }
     }
-    if ((int)threadIdx.x < a.k) {
-        const int32_t e = __ldg(a.topk_idx + mine + threadIdx.x);
+    if ((int)threadIdx.x < kK) {
+        const int32_t e = (int)threadIdx.x < a.k ? __ldg(a.topk_idx + mine + threadIdx.x) : -1;
         s_own[threadIdx.x] = (e >= 0 && e < a.E) ? e : -1;
     }
+    if constexpr (!kOwnInRegs)
+        __syncthreads();
+    // S <= kFusedMaxEntries, so entry indices fit in 32 bits; only the rounds
+    // that hold entries run, and a warp whose entries all lie past S skips them.
     uint32_t cnt[kK];
 #pragma unroll
     for (int j = 0; j < kK; ++j)
         cnt[j] = 0;
-    for (int64_t base = 0; base < S; base += (int64_t)nt * kFusedLoadRounds) {
+    const int32_t S32 = (int32_t)S, mine32 = (int32_t)mine;
+    for (int32_t base = 0; base < S32; base += nt * kFusedLoadRounds) {
         int32_t ev[kFusedLoadRounds];
 #pragma unroll
         for (int r = 0; r < kFusedLoadRounds; ++r) {
-            const int64_t i = base + (int64_t)r * nt + threadIdx.x;
-            ev[r] = i < S ? __ldg(a.topk_idx + i) : kNone;
+            const int32_t i = base + r * nt + (int32_t)threadIdx.x;
+            ev[r] = i < S32 ? __ldg(a.topk_idx + i) : kNone;
         }
 #pragma unroll
         for (int r = 0; r < kFusedLoadRounds; ++r) {
-            const int64_t i = base + (int64_t)r * nt + threadIdx.x;
+            const int32_t i = base + r * nt + (int32_t)threadIdx.x;
+            if (__all_sync(kFullMask, i >= S32))
+                break; // later rounds start further out
             const int32_t e = (ev[r] >= 0 && ev[r] < a.E) ? ev[r] : kNone;
+            const int32_t before = i - mine32; // entry i precedes (t, j) when before < j
 #pragma unroll
-            for (int j = 0; j < kK; ++j)
-                cnt[j] += (uint32_t)(e < own[j]) + ((uint32_t)(e == own[j] && i < mine + j) << 16);
+            for (int j = 0; j < kK; ++j) {
+                const int32_t o = kOwnInRegs ? own[kOwnInRegs ? j : 0] : s_own[j];
+                cnt[j] += e < o ? 1u : 0u;
+                cnt[j] += (e == o && before < j) ? 0x10000u : 0u;
+            }
         }
     }
 #pragma unroll
