@@ -452,6 +452,30 @@ def run_gpu(args, rank, world):
 EXPERT_INTERMEDIATE = 2048  # DeepSeek-V3 / Kimi-K2 routed-expert intermediate size
 
 
+def partial_accuracy(moe, d, wts, b, w, dev, sample=64):
+    """Errors of sender-side (per-rank partial) and receiver-only combine against
+    the fp64 weighted sum, on a sample of tokens: max and mean absolute error,
+    and the share of outputs where the two bf16 results differ."""
+    import torch
+    y_send = b["y"].view(torch.int16).cpu().numpy().view(np.uint16)
+    y_recv = moe.combine(d.handle, b["eo"]).view(torch.int16).cpu().numpy().view(np.uint16)
+    slot = d.handle.slot.cpu().numpy()
+    toks = np.linspace(0, w.T - 1, min(sample, w.T)).astype(np.int64)
+    to_f = lambda u: (u.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    sl = slot[toks]                                     # [n, k]
+    rows = torch.from_numpy(np.maximum(sl, 0).reshape(-1)).to(dev)
+    v = to_f(b["eo"].view(torch.int16)[rows].cpu().numpy().view(np.uint16)).reshape(len(toks), w.k, w.H)
+    wk = np.where(sl >= 0, wts[toks].astype(np.float64), 0.0)
+    exact = np.einsum("nk,nkh->nh", wk, v)
+    out = {}
+    for name, y in (("receiver", y_recv), ("sender", y_send)):
+        err = np.abs(to_f(y[toks]) - exact)
+        out[name] = {"max_abs": float(err.max()), "mean_abs": float(err.mean())}
+    out["differ_frac"] = float(np.mean(y_send[toks] != y_recv[toks]))
+    out["tokens"] = int(len(toks))
+    return out
+
+
 def run_op(args, peak, peak_kind):
     """Times one next-row kernel on a workload's shapes; prints one JSON line."""
     import math
@@ -531,7 +555,7 @@ def run_op(args, peak, peak_kind):
     if args.op == "rank_partial":
         npart = int(sets[0]["npart"].sum().item())
         nbytes = S * w.H * 2 + 2 * S * 4 + (w.R + 1) * 4 + 2 * npart * w.H * 2 + w.T * 4 + w.T * w.H * 2
-        extra = {"partials": npart}
+        extra = {"partials": npart, "accuracy": partial_accuracy(moe, d, wts, sets[0], w, dev)}
     elif args.op == "silu_quant":
         used = int((d.recv_src >= 0).sum().item())
         I = EXPERT_INTERMEDIATE

@@ -226,23 +226,14 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct(FusedArgs
 
     constexpr int L = kFusedLaneCols;
     const int32_t chunks = (a.H + chunk_cols<L>() - 1) / chunk_cols<L>();
-
-    // 1. The row's loads go out first: warp w owns chunks w, w + nwarps, ...
-    const uint16_t *xr = a.x + (int64_t)t * a.H;
-    LaneData<L> d[kChunks];
-#pragma unroll
-    for (int i = 0; i < kChunks; ++i) {
-        const int32_t c = warp + i * nwarps;
-        if (c < chunks)
-            load_chunk<L, kFp8>(xr, a.H, c, d[i]);
-    }
-
-    // 2. Own expert ids (broadcast loads) and this thread's share of all ids.
     const int64_t mine = (int64_t)t * a.k;
     constexpr int32_t kNone = 0x7fffffff; // never below or equal to a valid id
-    // Up to 8 own ids stay in registers; more are read from shared memory (the
-    // registers are needed for the row).
-    constexpr bool kOwnInRegs = kK <= 8;
+    const int32_t S32 = (int32_t)S, mine32 = (int32_t)mine; // S <= kFusedMaxEntries
+
+    // 1. The expert ids go out first (the own ids as broadcast loads, then this
+    //    thread's first round of all ids), ahead of the row, whose kilobytes
+    //    would otherwise queue in front of them.
+    constexpr bool kOwnInRegs = kK <= 8; // more own ids are read from shared memory
     int32_t own[kOwnInRegs ? kK : 1];
     if constexpr (kOwnInRegs) {
 #pragma unroll
@@ -251,25 +242,42 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct(FusedArgs
             own[j] = (e >= 0 && e < a.E) ? e : -1;
         }
     }
+    int32_t ev[kFusedLoadRounds];
+#pragma unroll
+    for (int r = 0; r < kFusedLoadRounds; ++r) {
+        const int32_t i = r * nt + (int32_t)threadIdx.x;
+        ev[r] = i < S32 ? __ldg(a.topk_idx + i) : kNone;
+    }
+
+    // 2. The row: warp w owns chunks w, w + nwarps, ...
+    const uint16_t *xr = a.x + (int64_t)t * a.H;
+    LaneData<L> d[kChunks];
+#pragma unroll
+    for (int i = 0; i < kChunks; ++i) {
+        const int32_t c = warp + i * nwarps;
+        if (c < chunks)
+            load_chunk<L, kFp8>(xr, a.H, c, d[i]);
+    }
     if ((int)threadIdx.x < kK) {
         const int32_t e = (int)threadIdx.x < a.k ? __ldg(a.topk_idx + mine + threadIdx.x) : -1;
         s_own[threadIdx.x] = (e >= 0 && e < a.E) ? e : -1;
     }
     if constexpr (!kOwnInRegs)
         __syncthreads();
-    // S <= kFusedMaxEntries, so entry indices fit in 32 bits; only the rounds
-    // that hold entries run, and a warp whose entries all lie past S skips them.
+
+    // 3. Counts of this thread's entries against the own ids, round by round;
+    //    a warp whose entries of a round all lie past S stops there.
     uint32_t cnt[kK];
 #pragma unroll
     for (int j = 0; j < kK; ++j)
         cnt[j] = 0;
-    const int32_t S32 = (int32_t)S, mine32 = (int32_t)mine;
     for (int32_t base = 0; base < S32; base += nt * kFusedLoadRounds) {
-        int32_t ev[kFusedLoadRounds];
+        if (base > 0) {
 #pragma unroll
-        for (int r = 0; r < kFusedLoadRounds; ++r) {
-            const int32_t i = base + r * nt + (int32_t)threadIdx.x;
-            ev[r] = i < S32 ? __ldg(a.topk_idx + i) : kNone;
+            for (int r = 0; r < kFusedLoadRounds; ++r) {
+                const int32_t i = base + r * nt + (int32_t)threadIdx.x;
+                ev[r] = i < S32 ? __ldg(a.topk_idx + i) : kNone;
+            }
         }
 #pragma unroll
         for (int r = 0; r < kFusedLoadRounds; ++r) {
@@ -294,7 +302,7 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct(FusedArgs
     }
     __syncthreads();
 
-    // 3. This token's slots: warp j adds the per-warp counts of entry j.
+    // 4. This token's slots: warp j adds the per-warp counts of entry j.
     for (int j = warp; j < a.k; j += nwarps) {
         const uint32_t v = (int)lane < nwarps ? s_part[lane][j] : 0u;
         const uint32_t tot = __reduce_add_sync(kFullMask, v);
@@ -313,14 +321,27 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct(FusedArgs
             s_slot[j] = s;
         }
     }
+
+    // 5. The row's codes, while the slot sums above complete.
+    LaneCodes<L> q[kFp8 ? kChunks : 1];
+    if constexpr (kFp8) {
+#pragma unroll
+        for (int i = 0; i < kChunks; ++i)
+            if (warp + i * nwarps < chunks)
+                quantise_lane<L>(d[i], q[i].codes, q[i].scale);
+    }
     __syncthreads();
 
-    // 4. Payload to the k slots.
+    // 6. Payload to the k slots.
 #pragma unroll
     for (int i = 0; i < kChunks; ++i) {
         const int32_t c = warp + i * nwarps;
-        if (c < chunks)
-            store_chunk<L, kFp8>(a.recv_x, a.recv_scale, a.H, c, a.k, s_slot, a.rows_cap, a.err, d[i]);
+        if (c >= chunks)
+            continue;
+        if constexpr (kFp8)
+            store_codes<L>(a.recv_x, a.recv_scale, a.H, c, a.k, s_slot, a.rows_cap, a.err, q[i]);
+        else
+            store_chunk<L, false>(a.recv_x, a.recv_scale, a.H, c, a.k, s_slot, a.rows_cap, a.err, d[i]);
     }
 }
 

@@ -18,10 +18,10 @@
 //  - fp8: lane l owns L consecutive columns, 128/L lanes make one 128-column
 //    block; the block's |x| maximum is reduced with butterfly shuffles inside
 //    those lanes, the scale is amax/448 and each code is e4m3(x/scale) with
-//    the binary32 quotient correctly rounded (see quotient_for_e4m3) and a
-//    saturating round-to-nearest-even conversion.  A lane stores its L codes with one L-byte store, and lane 0
-//    stores the warp's L/4 block scales with one store when the scale row
-//    allows it.
+//    the binary32 quotient correctly rounded (see product_decides_code) and a
+//    saturating round-to-nearest-even conversion.  A lane stores its L codes
+//    with one L-byte store, and lane 0 stores the warp's L/4 block scales with
+//    one store when the scale row allows it.
 // The token's k slots are read once per unit (lane j holds slot j) and
 // broadcast with shuffles.
 #pragma once
@@ -74,25 +74,19 @@ struct LaneData {
 // (>= 2^-6) and more than 3 units from such a boundary, both quotients give
 // the same code and q is used; otherwise (near a boundary, in the e4m3
 // subnormal range, a zero, or a block whose scale is below FLT_MIN) the exact
-// division is taken.  On N(0,1) data the slow branch is rare (~1e-4).
-__device__ __forceinline__ float quotient_for_e4m3(float x, float scale, float recip, bool fast)
+// division is taken.  On N(0,1) data the exact branch is rare (~1e-4 of the
+// values), so it is taken once per warp when any lane needs it.
+__device__ __forceinline__ bool product_decides_code(float q)
 {
-    if (fast) {
-        const float q = x * recip;
-        const uint32_t b = __float_as_uint(q) & 0x7fffffffu;
-        const int32_t off_mid = (int32_t)(b & 0xfffffu) - 0x80000;
-        if (b >= 0x3c800000u && (off_mid > 3 || off_mid < -3))
-            return q;
-    }
-    return __fdiv_rn(x, scale);
+    const uint32_t b = __float_as_uint(q) & 0x7fffffffu;
+    const uint32_t off_mid = ((b & 0xfffffu) - 0x7fffdu) & 0xfffffu; // <= 6: within 3 units of 0x80000
+    return b >= 0x3c800000u && off_mid > 6u;
 }
 
-// e4m3 codes of the lane's values, element 0 in the lowest byte, and the scale
-// of the lane's 128-column block.  All lanes of the warp call this together
-// (inactive lanes hold zeros).
-// e4m3 codes and the block scale of kLaneCols binary32 values per lane; the
-// 128/kLaneCols lanes of a 128-column block reduce the maximum together (all
-// lanes of the warp call this).
+// e4m3 codes (element 0 in the lowest byte) and the block scale of kLaneCols
+// binary32 values per lane; the 128/kLaneCols lanes of a 128-column block
+// reduce the maximum together.  All lanes of the warp call this (inactive lanes
+// hold zeros).  An all-zero block gets scale 0 and +0 codes.
 template <int kLaneCols>
 __device__ __forceinline__ void quantise_floats(const float (&f)[kLaneCols],
                                                 uint32_t (&codes)[kLaneCols / 4], float &scale_out)
@@ -104,24 +98,29 @@ __device__ __forceinline__ void quantise_floats(const float (&f)[kLaneCols],
 #pragma unroll
     for (int d = 64 / kLaneCols; d >= 1; d >>= 1)
         amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, d));
-    float scale = 0.0f;
+    const bool nonzero = amax > 0.0f;
+    const float scale = __fdiv_rn(nonzero ? amax : 448.0f, 448.0f);
+    const float recip = __frcp_rn(scale);
+    const bool fast = scale >= 0x1p-126f; // recip finite, products in range
+    float q[kLaneCols];
+    bool exact = !fast;
+#pragma unroll
+    for (int i = 0; i < kLaneCols; ++i) {
+        q[i] = f[i] * recip;
+        exact |= !product_decides_code(q[i]);
+    }
+    if (__any_sync(kFullMask, nonzero && exact)) {
+#pragma unroll
+        for (int i = 0; i < kLaneCols; ++i)
+            if (!fast || !product_decides_code(q[i]))
+                q[i] = __fdiv_rn(f[i], scale);
+    }
 #pragma unroll
     for (int i = 0; i < kLaneCols / 4; ++i)
-        codes[i] = 0u;
-    if (amax > 0.0f) {
-        scale = __fdiv_rn(amax, 448.0f);
-        const float recip = __frcp_rn(scale);
-        const bool fast = scale >= 0x1p-126f; // recip finite, products in range
-#pragma unroll
-        for (int i = 0; i < kLaneCols / 4; ++i) {
-            const float q0 = quotient_for_e4m3(f[4 * i + 0], scale, recip, fast);
-            const float q1 = quotient_for_e4m3(f[4 * i + 1], scale, recip, fast);
-            const float q2 = quotient_for_e4m3(f[4 * i + 2], scale, recip, fast);
-            const float q3 = quotient_for_e4m3(f[4 * i + 3], scale, recip, fast);
-            codes[i] = pack_e4m3x2(q0, q1) | (pack_e4m3x2(q2, q3) << 16);
-        }
-    }
-    scale_out = scale;
+        codes[i] = nonzero ? pack_e4m3x2(q[4 * i + 0], q[4 * i + 1]) |
+                                 (pack_e4m3x2(q[4 * i + 2], q[4 * i + 3]) << 16)
+                           : 0u;
+    scale_out = nonzero ? scale : 0.0f;
 }
 
 template <int kLaneCols>
@@ -166,9 +165,66 @@ __device__ __forceinline__ void load_chunk(const uint16_t *xr, int32_t H, int32_
     }
 }
 
+// e4m3 codes of the lane's columns of one chunk and its block's scale.
+template <int kLaneCols>
+struct LaneCodes {
+    uint32_t codes[kLaneCols / 4];
+    float scale;
+};
+
+// Stores quantised chunk c to the receive rows slots[0..k) of its token (-1 =
+// no row); the whole warp calls this.  `slots` may point to global or shared
+// memory.
+template <int kLaneCols>
+__device__ __forceinline__ void store_codes(void *recv_x, float *recv_scale, int32_t H, int32_t c,
+                                            int32_t k, const int32_t *slots, int64_t rows_cap,
+                                            int32_t *err, const LaneCodes<kLaneCols> &q)
+{
+    const unsigned lane = lane_id();
+    constexpr int kBlocks = chunk_cols<kLaneCols>() / 128; // scales per warp
+    constexpr int kLanesPerBlock = 128 / kLaneCols;
+    const int32_t nb = H / 128;
+    const int32_t col = lane_col<kLaneCols, true>(c, 0);
+    const bool active = col < H; // H % 128 == 0: whole blocks are in or out
+    float sc[kBlocks];
+#pragma unroll
+    for (int b = 0; b < kBlocks; ++b)
+        sc[b] = __shfl_sync(kFullMask, q.scale, b * kLanesPerBlock);
+    const bool scale_vec = (nb % kBlocks == 0) && (c * kBlocks + kBlocks - 1 < nb);
+    uint8_t *rx = static_cast<uint8_t *>(recv_x);
+    for (int32_t j0 = 0; j0 < k; j0 += kWarp) {
+        const int32_t my = j0 + (int32_t)lane < k ? checked_slot(slots[j0 + lane], rows_cap, err) : -1;
+        const int32_t jn = k - j0 < kWarp ? k - j0 : kWarp;
+        for (int32_t j = 0; j < jn; ++j) {
+            const int32_t s = __shfl_sync(kFullMask, my, j);
+            if (s < 0)
+                continue;
+            uint8_t *dst = rx + (int64_t)s * H + col;
+            if (active) {
+                if constexpr (kLaneCols == 16)
+                    st_v4(dst, make_uint4(q.codes[0], q.codes[1], q.codes[2], q.codes[3]));
+                else
+                    st_v2(dst, make_uint2(q.codes[0], q.codes[1]));
+            }
+            float *sr = recv_scale + (int64_t)s * nb;
+            if (scale_vec) {
+                if (lane == 0) {
+                    if constexpr (kBlocks == 4)
+                        st_v4(sr + c * 4, make_uint4(__float_as_uint(sc[0]), __float_as_uint(sc[1]),
+                                                     __float_as_uint(sc[2]), __float_as_uint(sc[3])));
+                    else
+                        st_v2(sr + c * 2, make_uint2(__float_as_uint(sc[0]), __float_as_uint(sc[1])));
+                }
+            } else if (active && lane % kLanesPerBlock == 0) {
+                sr[col / 128] = q.scale;
+            }
+        }
+    }
+}
+
 // Stores chunk c (loaded by load_chunk) to the receive rows slots[0..k) of its
-// token (-1 = no row); the whole warp calls this.  `slots` may point to global
-// or shared memory.
+// token (-1 = no row), quantising it first for fp8; the whole warp calls this.
+// `slots` may point to global or shared memory.
 template <int kLaneCols, bool kFp8>
 __device__ __forceinline__ void store_chunk(void *recv_x, float *recv_scale, int32_t H, int32_t c,
                                             int32_t k, const int32_t *slots, int64_t rows_cap,
@@ -176,49 +232,9 @@ __device__ __forceinline__ void store_chunk(void *recv_x, float *recv_scale, int
 {
     const unsigned lane = lane_id();
     if constexpr (kFp8) {
-        constexpr int kBlocks = chunk_cols<kLaneCols>() / 128; // scales per warp
-        constexpr int kLanesPerBlock = 128 / kLaneCols;
-        const int32_t nb = H / 128;
-        const int32_t col = lane_col<kLaneCols, true>(c, 0);
-        const bool active = col < H; // H % 128 == 0: whole blocks are in or out
-        uint32_t codes[kLaneCols / 4];
-        float scale;
-        quantise_lane<kLaneCols>(d, codes, scale);
-        float sc[kBlocks];
-#pragma unroll
-        for (int b = 0; b < kBlocks; ++b)
-            sc[b] = __shfl_sync(kFullMask, scale, b * kLanesPerBlock);
-        const bool scale_vec = (nb % kBlocks == 0) && (c * kBlocks + kBlocks - 1 < nb);
-        uint8_t *rx = static_cast<uint8_t *>(recv_x);
-        for (int32_t j0 = 0; j0 < k; j0 += kWarp) {
-            const int32_t my =
-                j0 + (int32_t)lane < k ? checked_slot(slots[j0 + lane], rows_cap, err) : -1;
-            const int32_t jn = k - j0 < kWarp ? k - j0 : kWarp;
-            for (int32_t j = 0; j < jn; ++j) {
-                const int32_t s = __shfl_sync(kFullMask, my, j);
-                if (s < 0)
-                    continue;
-                uint8_t *dst = rx + (int64_t)s * H + col;
-                if (active) {
-                    if constexpr (kLaneCols == 16)
-                        st_v4(dst, make_uint4(codes[0], codes[1], codes[2], codes[3]));
-                    else
-                        st_v2(dst, make_uint2(codes[0], codes[1]));
-                }
-                float *sr = recv_scale + (int64_t)s * nb;
-                if (scale_vec) {
-                    if (lane == 0) {
-                        if constexpr (kBlocks == 4)
-                            st_v4(sr + c * 4, make_uint4(__float_as_uint(sc[0]), __float_as_uint(sc[1]),
-                                                         __float_as_uint(sc[2]), __float_as_uint(sc[3])));
-                        else
-                            st_v2(sr + c * 2, make_uint2(__float_as_uint(sc[0]), __float_as_uint(sc[1])));
-                    }
-                } else if (active && lane % kLanesPerBlock == 0) {
-                    sr[col / 128] = scale;
-                }
-            }
-        }
+        LaneCodes<kLaneCols> q;
+        quantise_lane<kLaneCols>(d, q.codes, q.scale);
+        store_codes<kLaneCols>(recv_x, recv_scale, H, c, k, slots, rows_cap, err, q);
     } else {
         uint16_t *rx = static_cast<uint16_t *>(recv_x);
         for (int32_t j0 = 0; j0 < k; j0 += kWarp) {
