@@ -565,6 +565,9 @@ def run_op(args, peak, peak_kind):
         nbytes = w.T * w.E * 4 + S * 8
         extra = {}
     gbs = nbytes / (us * 1e-6) / 1e9
+    op_kernels = {"rank_partial": ["combine_partial_send", "combine_partial_recv"],
+                  "silu_quant": ["silu_quant_rows"], "router": ["router_topk"]}[args.op]
+    extra["traffic"] = {k: recorded_traffic(k, w.name) for k in op_kernels}
     line = {"op": args.op, "workload": w.name, "us": round(us, 3), "algorithmic_bytes": nbytes,
             "achieved_GBs": round(gbs, 1), "peak": peak, "peak_kind": peak_kind,
             "frac": round(gbs / peak, 4), "launches_timed": launches,
