@@ -523,6 +523,17 @@ def run_op(args, peak, peak_kind):
         fn = lambda b: (lambda: moe.router_topk_into(b["l"], w.k, b["idx"], b["w"],
                                                      score_fn="sigmoid" if w.routing == "sigmoid_topk" else "softmax",
                                                      stream=stream))
+    elif args.op == "route_dispatch":
+        logits = torch.from_numpy(np.random.default_rng(w.seed).standard_normal((w.T, w.E)).astype(np.float32)).to(dev)
+        cfg = moe.make_config(w.H, w.k, w.E, w.R, w.fp8, w.pad128)
+        x_dev = bf16_dev(x)
+        set_bytes = w.T * w.E * 4 + sum(algorithmic_bytes(w.T, w.H, w.E, w.R, w.k, w.fp8)[:1])
+        make = lambda: dict(l=logits.clone(), x=x_dev.clone(), buf=moe.Buffers(cfg, w.T, dev),
+                            idx=torch.empty((w.T, w.k), dtype=torch.int32, device=dev),
+                            w=torch.empty((w.T, w.k), dtype=torch.float32, device=dev))
+        fn = lambda b: (lambda: moe.route_dispatch_into(
+            b["buf"], b["x"], b["l"], b["idx"], b["w"],
+            score_fn="sigmoid" if w.routing == "sigmoid_topk" else "softmax", stream=stream))
     else:
         raise SystemExit(f"unknown --op {args.op}")
     nsets = 1 if set_bytes >= 2 * l2 else min(64, math.ceil(2 * l2 / set_bytes) + 1)
@@ -561,12 +572,17 @@ def run_op(args, peak, peak_kind):
         I = EXPERT_INTERMEDIATE
         nbytes = used * (4 * I + I + (I // 128) * 4) + used * 4
         extra = {"rows_used": used, "I": I}
+    elif args.op == "route_dispatch":
+        nbytes = w.T * w.E * 4 + S * 8 + algorithmic_bytes(w.T, w.H, w.E, w.R, w.k, w.fp8)[0]
+        extra = {}
     else:
         nbytes = w.T * w.E * 4 + S * 8
         extra = {}
     gbs = nbytes / (us * 1e-6) / 1e9
     op_kernels = {"rank_partial": ["combine_partial_send", "combine_partial_recv"],
-                  "silu_quant": ["silu_quant_rows"], "router": ["router_topk"]}[args.op]
+                  "silu_quant": ["silu_quant_rows"], "router": ["router_topk"],
+                  "route_dispatch": ["router_topk", "dispatch_direct", "dispatch_fused",
+                                     "scatter_rows", "scatter_bulk_bf16"]}[args.op]
     extra["traffic"] = {k: recorded_traffic(k, w.name) for k in op_kernels}
     line = {"op": args.op, "workload": w.name, "us": round(us, 3), "algorithmic_bytes": nbytes,
             "achieved_GBs": round(gbs, 1), "peak": peak, "peak_kind": peak_kind,
@@ -583,7 +599,7 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", default=None, choices=["rank_partial", "silu_quant", "router"],
+    ap.add_argument("--op", default=None, choices=["rank_partial", "silu_quant", "router", "route_dispatch"],
                     help="time one of the kernels next to the hot path instead of the step")
     args = ap.parse_args()
     if args.warmup < 3:

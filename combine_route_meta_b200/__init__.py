@@ -109,6 +109,10 @@ def _declare(lib):
     lib.moe_silu_quant.restype = ctypes.c_int
     lib.moe_router_topk.argtypes = [i32, i32, i32, P, i32, i32, i32, i32, P, P, P]
     lib.moe_router_topk.restype = ctypes.c_int
+    lib.moe_route_dispatch.argtypes = [cfgp, i32, P, P, i32, i32, i32, i32, P, P,
+                                       ctypes.POINTER(moe_dispatch_out), P, P, ctypes.c_size_t, P, P,
+                                       ctypes.POINTER(moe_handle)]
+    lib.moe_route_dispatch.restype = ctypes.c_int
     lib.moe_check.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
     lib.moe_check.restype = ctypes.c_int
     return lib
@@ -132,6 +136,7 @@ moe_selftest_bounded_wait = lib.moe_selftest_bounded_wait
 moe_combine_rank_partial = lib.moe_combine_rank_partial
 moe_silu_quant = lib.moe_silu_quant
 moe_router_topk = lib.moe_router_topk
+moe_route_dispatch = lib.moe_route_dispatch
 
 
 class MoeError(RuntimeError):
@@ -404,3 +409,40 @@ def router_topk(logits: torch.Tensor, k: int, **kw):
     w = torch.empty((T, k), dtype=torch.float32, device=logits.device)
     router_topk_into(logits.contiguous().float(), k, idx, w, **kw)
     return idx, w
+
+
+def route_dispatch_into(buf: Buffers, x: torch.Tensor, logits: torch.Tensor, topk_idx: torch.Tensor,
+                        topk_w: torch.Tensor, *, score_fn: str = "softmax", n_group: int = 1,
+                        topk_group: int = 1, renormalize: bool = True,
+                        stream: Optional[torch.cuda.Stream] = None) -> None:
+    """moe_route_dispatch into preallocated buffers: the router writes topk_idx
+    and topk_w, then the dispatch reads them."""
+    P = ctypes.c_void_p
+    st = lib.moe_route_dispatch(ctypes.byref(buf.cfg), buf.T, P(x.data_ptr()), P(logits.data_ptr()),
+                                {"softmax": SCORE_SOFTMAX, "sigmoid": SCORE_SIGMOID}[score_fn],
+                                n_group, topk_group, 1 if renormalize else 0,
+                                P(topk_idx.data_ptr()), P(topk_w.data_ptr()), ctypes.byref(buf.out),
+                                P(buf.slot.data_ptr()), P(buf.workspace.data_ptr()), buf.workspace_bytes,
+                                P(buf.err.data_ptr()), P(_stream_ptr(stream)), ctypes.byref(buf.handle_c))
+    _ok(st, "moe_route_dispatch")
+
+
+def route_dispatch(x: torch.Tensor, logits: torch.Tensor, k: int, num_experts: int,
+                   num_virtual_ranks: int, fp8: bool, pad128: bool = False, *,
+                   stream: Optional[torch.cuda.Stream] = None, **router_kw):
+    """Router top-k on logits[T,E] (float32), then dispatch of x[T,H] (bf16).
+
+    Returns (DispatchResult, topk_idx, topk_w); the handle keeps topk_w."""
+    _check_tensor(x, "x", torch.bfloat16, 2)
+    _check_tensor(logits, "logits", torch.float32, 2)
+    T, H = x.shape
+    if logits.shape != (T, num_experts):
+        raise ValueError("logits must be [T, num_experts]")
+    cfg = make_config(H, k, num_experts, num_virtual_ranks, fp8, pad128)
+    buf = Buffers(cfg, T, x.device)
+    idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
+    w = torch.empty((T, k), dtype=torch.float32, device=x.device)
+    route_dispatch_into(buf, x, logits, idx, w, stream=stream, **router_kw)
+    handle = Handle(buf.handle_c, buf.slot, w)
+    return (DispatchResult(buf.recv_x, buf.recv_scale, buf.expert_count, buf.expert_offset,
+                           buf.rank_offset, buf.recv_src, handle), idx, w)

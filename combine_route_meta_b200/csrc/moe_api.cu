@@ -189,49 +189,79 @@ int fused_chunks(const moe_config *c, int32_t T, unsigned *threads)
     return 0;
 }
 
-template <bool kFp8>
-cudaError_t launch_fused(int per, unsigned grid, unsigned block, size_t smem, cudaStream_t s,
-                         const FusedArgs &f)
+using SmallKernel = void (*)(FusedArgs);
+
+// The one-token-per-CTA dispatch kernel for a shape: the direct-rank form
+// without padding, the histogram form with it.
+SmallKernel small_kernel(bool fp8, bool pad, bool big_k, int per)
 {
-    switch (per) {
-    case 1:
-        return launch(dispatch_fused<1, kFp8>, grid, block, smem, s, f);
-    case 2:
-        return launch(dispatch_fused<2, kFp8>, grid, block, smem, s, f);
-    default:
-        return launch(dispatch_fused<4, kFp8>, grid, block, smem, s, f);
+    const int i = per == 1 ? 0 : (per == 2 ? 1 : 2);
+    if (pad) {
+        static const SmallKernel t[2][3] = {
+            {dispatch_fused<1, false>, dispatch_fused<2, false>, dispatch_fused<4, false>},
+            {dispatch_fused<1, true>, dispatch_fused<2, true>, dispatch_fused<4, true>}};
+        return t[fp8][i];
     }
+    static const SmallKernel t[2][2][3] = {
+        {{dispatch_direct<1, false, 8>, dispatch_direct<2, false, 8>, dispatch_direct<4, false, 8>},
+         {dispatch_direct<1, false, kFusedMaxK>, dispatch_direct<2, false, kFusedMaxK>,
+          dispatch_direct<4, false, kFusedMaxK>}},
+        {{dispatch_direct<1, true, 8>, dispatch_direct<2, true, 8>, dispatch_direct<4, true, 8>},
+         {dispatch_direct<1, true, kFusedMaxK>, dispatch_direct<2, true, kFusedMaxK>,
+          dispatch_direct<4, true, kFusedMaxK>}}};
+    return t[fp8][big_k][i];
 }
 
-template <bool kFp8, int kK>
-cudaError_t launch_direct_k(int per, unsigned grid, unsigned block, size_t smem, cudaStream_t s,
-                            const FusedArgs &f)
+// Resident CTAs per SM of a kernel at a block size, cached per device.
+int cached_per_sm(const void *fn, int block, size_t smem)
 {
-    switch (per) {
-    case 1:
-        return launch(dispatch_direct<1, kFp8, kK>, grid, block, smem, s, f);
-    case 2:
-        return launch(dispatch_direct<2, kFp8, kK>, grid, block, smem, s, f);
-    default:
-        return launch(dispatch_direct<4, kFp8, kK>, grid, block, smem, s, f);
-    }
+    struct Entry {
+        const void *fn;
+        int block, dev, n;
+        size_t smem;
+    };
+    static Entry cache[256];
+    static int used = 0;
+    static std::mutex m;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return 0;
+    std::lock_guard<std::mutex> lock(m);
+    for (int i = 0; i < used; ++i)
+        if (cache[i].fn == fn && cache[i].block == block && cache[i].smem == smem && cache[i].dev == dev)
+            return cache[i].n;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, block, smem) != cudaSuccess || n <= 0)
+        return 0;
+    if (used < 256)
+        cache[used++] = Entry{fn, block, dev, n, smem};
+    return n;
 }
 
-// The fused dispatch of one token per CTA: the direct-rank form without
-// padding (T token CTAs and one metadata CTA), the histogram form with it.
-cudaError_t launch_small(bool fp8, int per, int32_t T, unsigned block, cudaStream_t s,
-                         const FusedArgs &f)
+// Launches the one-token-per-CTA dispatch.  Chunks per warp start at `per`
+// (the fewest that fit the row in one CTA) and grow while the grid would not
+// be resident in one wave: at T near or above the SM count, two CTAs of half
+// the warps per SM beat two waves of one.
+cudaError_t launch_small(bool fp8, int per, int32_t T, int sms, cudaStream_t s, const FusedArgs &f)
 {
     const size_t smem = fused_smem(f.E);
-    if (f.pad128)
-        return fp8 ? launch_fused<true>(per, T, block, smem, s, f)
-                   : launch_fused<false>(per, T, block, smem, s, f);
-    const unsigned grid = (unsigned)T + 1;
-    if (f.k <= 8)
-        return fp8 ? launch_direct_k<true, 8>(per, grid, block, smem, s, f)
-                   : launch_direct_k<false, 8>(per, grid, block, smem, s, f);
-    return fp8 ? launch_direct_k<true, kFusedMaxK>(per, grid, block, smem, s, f)
-               : launch_direct_k<false, kFusedMaxK>(per, grid, block, smem, s, f);
+    const bool pad = f.pad128 != 0;
+    const bool big_k = f.k > 8;
+    const unsigned grid = pad ? (unsigned)T : (unsigned)T + 1;
+    const int32_t chunks = (f.H + chunk_cols<kFusedLaneCols>() - 1) / chunk_cols<kFusedLaneCols>();
+    int chosen = per;
+    for (int p = per; p <= kFusedMaxChunks; p *= 2) {
+        const int block = (chunks + p - 1) / p * kWarp;
+        const int n = cached_per_sm((const void *)small_kernel(fp8, pad, big_k, p), block, smem);
+        if (n == 0)
+            return cudaErrorInvalidConfiguration;
+        if ((int64_t)grid <= (int64_t)sms * n) {
+            chosen = p;
+            break;
+        }
+    }
+    const unsigned block = (unsigned)((chunks + chosen - 1) / chosen * kWarp);
+    return launch(small_kernel(fp8, pad, big_k, chosen), grid, block, smem, s, f);
 }
 
 size_t workspace_bytes(const moe_config *c, int32_t T)
@@ -431,10 +461,12 @@ int moe_dispatch_sizes_for(const moe_config *cfg, int32_t T, int64_t rows_cap,
     return MOE_OK;
 }
 
-int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t *topk_idx,
-                 const float *topk_w, const moe_dispatch_out *out, int32_t *slot,
-                 void *workspace, size_t workspace_bytes_given, int32_t *dev_err, void *stream,
-                 moe_handle *handle)
+namespace {
+
+int check_dispatch_args(const moe_config *cfg, int32_t T, const void *x, const int32_t *topk_idx,
+                        const float *topk_w, const moe_dispatch_out *out, int32_t *slot,
+                        void *workspace, size_t workspace_bytes_given, int32_t *dev_err,
+                        moe_handle *handle)
 {
     int st = check_config(cfg);
     if (st != MOE_OK)
@@ -445,10 +477,112 @@ int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
                                 dev_err)) != MOE_OK ||
         (st = check_payload_args(cfg, T, x, slot, out)) != MOE_OK)
         return st;
+    return MOE_OK;
+}
+
+// Checks of moe_router_topk's arguments (T == 0 passes).
+int check_router_args(int32_t T, int32_t E, int32_t k, const float *logits, int32_t score_fn,
+                      int32_t n_group, int32_t topk_group, const int32_t *topk_idx,
+                      const float *topk_w)
+{
+    if (T < 0 || E <= 0 || k <= 0 || n_group <= 0 || topk_group <= 0 || topk_group > n_group ||
+        (score_fn != MOE_SCORE_SOFTMAX && score_fn != MOE_SCORE_SIGMOID) || E % n_group != 0)
+        return MOE_ERR_INVALID_ARG;
+    if ((int64_t)k > (int64_t)topk_group * (E / n_group))
+        return MOE_ERR_INVALID_ARG;
+    if (E > kRouterMaxE || k > kRouterMaxK || n_group > kRouterMaxGroups)
+        return MOE_ERR_UNSUPPORTED;
+    if (T > 0 && (logits == nullptr || topk_idx == nullptr || topk_w == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+int launch_router(int32_t T, int32_t E, int32_t k, const float *logits, int32_t score_fn,
+                  int32_t n_group, int32_t topk_group, int32_t renormalize, int32_t *topk_idx,
+                  float *topk_w, const DeviceInfo *dev, cudaStream_t s)
+{
+    RouterArgs a;
+    a.logits = logits;
+    a.T = T;
+    a.E = E;
+    a.k = k;
+    a.score_fn = score_fn;
+    a.n_group = n_group;
+    a.topk_group = topk_group;
+    a.renormalize = renormalize ? 1 : 0;
+    a.topk_idx = topk_idx;
+    a.topk_w = topk_w;
+    const unsigned block = kRouterWarps * kWarp;
+    const int64_t units = (T + kRouterWarps - 1) / kRouterWarps;
+    // logits per lane, rounded up to a power of two; at most one wave of CTAs
+    if (E <= 4 * kWarp)
+        return launched(launch(router_topk<4>, grid_for(units, dev->sms, dev->router_per_sm[0]),
+                               block, 0, s, a));
+    if (E <= 8 * kWarp)
+        return launched(launch(router_topk<8>, grid_for(units, dev->sms, dev->router_per_sm[1]),
+                               block, 0, s, a));
+    if (E <= 16 * kWarp)
+        return launched(launch(router_topk<16>, grid_for(units, dev->sms, dev->router_per_sm[2]),
+                               block, 0, s, a));
+    return launched(launch(router_topk<kRouterMaxE / kWarp>,
+                           grid_for(units, dev->sms, dev->router_per_sm[3]), block, 0, s, a));
+}
+
+int run_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t *topk_idx,
+                 const float *topk_w, const moe_dispatch_out *out, int32_t *slot,
+                 void *workspace, int32_t *dev_err, DeviceInfo *dev, cudaStream_t s,
+                 moe_handle *handle);
+
+} // namespace
+
+int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t *topk_idx,
+                 const float *topk_w, const moe_dispatch_out *out, int32_t *slot,
+                 void *workspace, size_t workspace_bytes_given, int32_t *dev_err, void *stream,
+                 moe_handle *handle)
+{
+    int st = check_dispatch_args(cfg, T, x, topk_idx, topk_w, out, slot, workspace,
+                                 workspace_bytes_given, dev_err, handle);
+    if (st != MOE_OK)
+        return st;
+    DeviceInfo *dev = nullptr;
+    if ((st = device_info(&dev)) != MOE_OK)
+        return st;
+    return run_dispatch(cfg, T, x, topk_idx, topk_w, out, slot, workspace, dev_err, dev,
+                        static_cast<cudaStream_t>(stream), handle);
+}
+
+int moe_route_dispatch(const moe_config *cfg, int32_t T, const void *x, const float *logits,
+                       int32_t score_fn, int32_t n_group, int32_t topk_group, int32_t renormalize,
+                       int32_t *topk_idx, float *topk_w, const moe_dispatch_out *out,
+                       int32_t *slot, void *workspace, size_t workspace_bytes_given,
+                       int32_t *dev_err, void *stream, moe_handle *handle)
+{
+    int st = check_config(cfg);
+    if (st != MOE_OK)
+        return st;
+    if ((st = check_router_args(T, cfg->E, cfg->k, logits, score_fn, n_group, topk_group, topk_idx,
+                                topk_w)) != MOE_OK ||
+        (st = check_dispatch_args(cfg, T, x, topk_idx, topk_w, out, slot, workspace,
+                                  workspace_bytes_given, dev_err, handle)) != MOE_OK)
+        return st;
     DeviceInfo *dev = nullptr;
     if ((st = device_info(&dev)) != MOE_OK)
         return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T > 0 && (st = launch_router(T, cfg->E, cfg->k, logits, score_fn, n_group, topk_group,
+                                     renormalize, topk_idx, topk_w, dev, s)) != MOE_OK)
+        return st;
+    return run_dispatch(cfg, T, x, topk_idx, topk_w, out, slot, workspace, dev_err, dev, s, handle);
+}
+
+namespace {
+
+int run_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t *topk_idx,
+                 const float *topk_w, const moe_dispatch_out *out, int32_t *slot,
+                 void *workspace, int32_t *dev_err, DeviceInfo *dev, cudaStream_t s,
+                 moe_handle *handle)
+{
+    int st;
     const bool fp8 = cfg->flags & MOE_FP8;
 
     unsigned fused_block = 0;
@@ -471,7 +605,7 @@ int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
         f.recv_src = out->recv_src;
         f.slot = slot;
         f.err = dev_err;
-        const cudaError_t e = launch_small(fp8, per, T, fused_block, s, f);
+        const cudaError_t e = launch_small(fp8, per, T, dev->sms, s, f);
         if ((st = launched(e)) != MOE_OK)
             return st;
     } else {
@@ -486,6 +620,8 @@ int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
     handle->rows_cap = out->rows_cap;
     return MOE_OK;
 }
+
+} // namespace
 
 int moe_dispatch_layout(const moe_config *cfg, int32_t T, const int32_t *topk_idx,
                         const moe_dispatch_out *out, int32_t *slot, void *workspace,
@@ -677,47 +813,14 @@ int moe_router_topk(int32_t T, int32_t E, int32_t k, const float *logits, int32_
                     int32_t n_group, int32_t topk_group, int32_t renormalize, int32_t *topk_idx,
                     float *topk_w, void *stream)
 {
-    if (T < 0 || E <= 0 || k <= 0 || n_group <= 0 || topk_group <= 0 || topk_group > n_group ||
-        (score_fn != MOE_SCORE_SOFTMAX && score_fn != MOE_SCORE_SIGMOID) || E % n_group != 0)
-        return MOE_ERR_INVALID_ARG;
-    if ((int64_t)k > (int64_t)topk_group * (E / n_group))
-        return MOE_ERR_INVALID_ARG;
-    if (E > kRouterMaxE || k > kRouterMaxK || n_group > kRouterMaxGroups)
-        return MOE_ERR_UNSUPPORTED;
-    if (T == 0)
-        return MOE_OK;
-    if (logits == nullptr || topk_idx == nullptr || topk_w == nullptr)
-        return MOE_ERR_INVALID_ARG;
+    int st = check_router_args(T, E, k, logits, score_fn, n_group, topk_group, topk_idx, topk_w);
+    if (st != MOE_OK || T == 0)
+        return st;
     DeviceInfo *dev = nullptr;
-    int st;
     if ((st = device_info(&dev)) != MOE_OK)
         return st;
-    RouterArgs a;
-    a.logits = logits;
-    a.T = T;
-    a.E = E;
-    a.k = k;
-    a.score_fn = score_fn;
-    a.n_group = n_group;
-    a.topk_group = topk_group;
-    a.renormalize = renormalize ? 1 : 0;
-    a.topk_idx = topk_idx;
-    a.topk_w = topk_w;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const unsigned block = kRouterWarps * kWarp;
-    const int64_t units = (T + kRouterWarps - 1) / kRouterWarps;
-    // logits per lane, rounded up to a power of two; at most one wave of CTAs
-    if (E <= 4 * kWarp)
-        return launched(launch(router_topk<4>, grid_for(units, dev->sms, dev->router_per_sm[0]),
-                               block, 0, s, a));
-    if (E <= 8 * kWarp)
-        return launched(launch(router_topk<8>, grid_for(units, dev->sms, dev->router_per_sm[1]),
-                               block, 0, s, a));
-    if (E <= 16 * kWarp)
-        return launched(launch(router_topk<16>, grid_for(units, dev->sms, dev->router_per_sm[2]),
-                               block, 0, s, a));
-    return launched(launch(router_topk<kRouterMaxE / kWarp>,
-                           grid_for(units, dev->sms, dev->router_per_sm[3]), block, 0, s, a));
+    return launch_router(T, E, k, logits, score_fn, n_group, topk_group, renormalize, topk_idx,
+                         topk_w, dev, static_cast<cudaStream_t>(stream));
 }
 
 int moe_check(int32_t *dev_err, void *stream, int32_t *bits_out)

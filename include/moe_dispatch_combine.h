@@ -308,6 +308,24 @@ MOE_API int moe_router_topk(int32_t T, int32_t E, int32_t k, const float *logits
                             int32_t renormalize, int32_t *topk_idx, float *topk_w, void *stream);
 
 /*
+ * Router top-k followed by dispatch, in one call: moe_router_topk on logits[T,
+ * E] (E = cfg->E, k = cfg->k) writes topk_idx[T, k] and topk_w[T, k], and
+ * moe_dispatch then reads them ("Lower latency and higher throughput with
+ * multi-node DeepSeek deployment", section "Roteador MoE": the router is the
+ * step right before dispatch).  The two kernels are stream-ordered and the
+ * second starts launching while the first finishes; the ids and weights
+ * (a few KB at decode sizes) are read back from L2.  Every argument of both
+ * steps is checked before anything is enqueued; results, errors and the
+ * handle are those of the two calls made one after the other.
+ */
+MOE_API int moe_route_dispatch(const moe_config *cfg, int32_t T, const void *x,
+                               const float *logits, int32_t score_fn, int32_t n_group,
+                               int32_t topk_group, int32_t renormalize, int32_t *topk_idx,
+                               float *topk_w, const moe_dispatch_out *out, int32_t *slot,
+                               void *workspace, size_t workspace_bytes, int32_t *dev_err,
+                               void *stream, moe_handle *handle);
+
+/*
  * moe_dispatch without a workspace argument, for callers that cannot allocate
  * device memory (the pages have no counterpart; this is a deployment aid).
  *

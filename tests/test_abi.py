@@ -94,6 +94,26 @@ def test_dispatch_rejects_bad_arguments_before_touching_the_gpu():
                             None, 0, P(16), None, ctypes.byref(h)) == moe.ERR_INVALID_ARG
 
 
+def test_route_dispatch_checks_both_steps_before_launching():
+    # every case fails a check of the router or of the dispatch, so nothing runs
+    cfg = moe.make_config(256, 2, 8, 2, fp8=False)
+    out = moe.moe_dispatch_out(16, None, 16, 16, 16, 16, 32)
+    h = moe.moe_handle()
+    P = ctypes.c_void_p
+    def call(c=cfg, T=16, logits=P(16), fn=moe.SCORE_SOFTMAX, G=1, TG=1, err=P(16), x=P(16)):
+        return moe.moe_route_dispatch(ctypes.byref(c), T, x, logits, fn, G, TG, 1, P(16), P(16),
+                                      ctypes.byref(out), P(16), None, 0, err, None, ctypes.byref(h))
+    assert call(logits=None) == moe.ERR_INVALID_ARG          # router: no logits
+    assert call(fn=7) == moe.ERR_INVALID_ARG                  # router: unknown score function
+    assert call(G=3) == moe.ERR_INVALID_ARG                   # router: groups do not divide E
+    assert call(G=8, TG=1) == moe.ERR_INVALID_ARG             # router: k > topk_group * E / n_group
+    assert call(err=None) == moe.ERR_INVALID_ARG              # dispatch: no error word
+    assert call(x=P(18)) == moe.ERR_INVALID_ARG               # dispatch: misaligned x
+    assert call(T=-1) == moe.ERR_INVALID_ARG
+    wide = moe.make_config(256, 2, 2048, 2, fp8=False)        # E beyond the router's limit
+    assert call(c=wide) == moe.ERR_UNSUPPORTED
+
+
 def test_combine_rejects_bad_arguments():
     h = moe.moe_handle(moe.make_config(256, 2, 8, 2, False), 16, 16, 16, 32)
     P = ctypes.c_void_p

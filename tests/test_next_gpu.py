@@ -179,3 +179,33 @@ def test_router_topk_ties_zeros_and_infinities(E, G, TG, fn):
     idx, w = moe.router_topk(to_dev(l), k, score_fn=fn, n_group=G, topk_group=TG, renormalize=True)
     np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
     np.testing.assert_allclose(w.cpu().numpy(), ref_w, rtol=2e-6, atol=1e-9)
+
+
+# ---- router feeding dispatch in one call ------------------------------------------------
+
+@pytest.mark.parametrize("T,E,R,k,H,fn,G,TG,fp8,pad", [
+    (128, 256, 8, 8, 7168, "sigmoid", 8, 4, True, False),   # DeepSeek-V3-shaped decode
+    (16, 8, 2, 2, 256, "softmax", 1, 1, False, False),
+    (3000, 256, 32, 8, 512, "softmax", 1, 1, True, True),   # tiled metadata path
+])
+def test_route_dispatch_equals_router_then_dispatch(T, E, R, k, H, fn, G, TG, fp8, pad):
+    rng = np.random.default_rng(T + E)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    x = f32_to_bf16_bits(rng.standard_normal((T, H)).astype(np.float32))
+    d, idx, w = moe.route_dispatch(bf16_to_dev(x), to_dev(logits), k, E, R, fp8, pad,
+                                   score_fn=fn, n_group=G, topk_group=TG)
+    assert moe.check() == 0
+    ref_idx, ref_w = oracle.router_topk(logits, k, score_fn=fn, n_group=G, topk_group=TG)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
+    np.testing.assert_allclose(w.cpu().numpy(), ref_w, rtol=2e-6, atol=1e-9)
+    d2 = moe.dispatch(bf16_to_dev(x), idx.clone(), w.clone(), E, R, fp8, pad)
+    for a, b in [(d.expert_count, d2.expert_count), (d.expert_offset, d2.expert_offset),
+                 (d.rank_offset, d2.rank_offset), (d.handle.slot, d2.handle.slot)]:
+        np.testing.assert_array_equal(a.cpu().numpy(), b.cpu().numpy())
+    n = int(d.expert_offset[E].item())
+    np.testing.assert_array_equal(d.recv_src[:n].cpu().numpy(), d2.recv_src[:n].cpu().numpy())
+    valid = d.recv_src[:n] >= 0
+    np.testing.assert_array_equal(d.recv_x[:n][valid].view(torch.uint8).cpu().numpy(),
+                                  d2.recv_x[:n][valid].view(torch.uint8).cpu().numpy())
+    o = oracle.dispatch(x, ref_idx, E=E, R=R, fp8=fp8, pad128=pad)
+    np.testing.assert_array_equal(d.handle.slot.cpu().numpy(), o["slot"])

@@ -168,6 +168,13 @@ CASES = [
     (3, 16384, 16, 4, 4, True, False, True),
     (2, 24576, 16, 4, 4, True, True, True),
     (256, 7168, 256, 32, 8, True, True, True),   # S = 2048: the largest fused batch
+    # around one resident wave of token CTAs (148 SMs): the launch doubles the
+    # chunks per warp when T (+1) CTAs of one chunk would need two waves
+    (147, 7168, 256, 8, 8, True, False, True),
+    (148, 7168, 256, 8, 8, False, False, True),
+    (149, 7168, 256, 8, 8, True, True, True),
+    (256, 7168, 256, 8, 8, True, False, True),
+    (170, 4096, 128, 8, 12, True, False, False), # k > 8 own ids from shared memory, duplicates
     # one-CTA metadata + scatter: k > 16, or 2048 < S <= 4096
     (10, 128, 8, 2, 20, False, False, False),
     (600, 1032, 16, 4, 5, False, True, False),   # ragged last 512-column chunk (8 columns)
