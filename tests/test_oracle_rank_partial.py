@@ -44,6 +44,19 @@ def test_partial_rounding_is_nearest_even_bf16():
         assert o["partial"][0, 0, 0] == _nearest_bf16_exact(float(np.float32(w)))
 
 
+def test_partial_rounding_ties_go_to_even():
+    # weights whose low 16 bits are exactly 0x8000 sit halfway between two bf16
+    # values: the partial takes the one with an even last bit
+    idx = np.zeros((1, 1), np.int32)
+    slot = np.zeros((1, 1), np.int32)
+    eo = np.full((1, 4), 0x3F80, np.uint16)  # 1.0
+    for bits, want in [(0x3F808000, 0x3F80), (0x3F818000, 0x3F82), (0xBF808000, 0xBF80),
+                       (0xBF818000, 0xBF82), (0x40A78000, 0x40A8), (0x3C008000, 0x3C00)]:
+        w = np.array([[bits]], np.uint32).view(np.float32)
+        o = oracle.combine_rank_partial(idx, slot, w, eo, E=1, R=1)
+        assert o["partial"][0, 0, 0] == want == _nearest_bf16_exact(float(w[0, 0])), hex(bits)
+
+
 def test_one_rank_equals_receiver_sum_rounded_once():
     x, idx, w = random_problem(4, 30, 64, 8, 4)
     d = oracle.dispatch(x, idx, E=8, R=1, fp8=False)

@@ -55,6 +55,18 @@ def test_group_limited_invariants():
         np.testing.assert_allclose(w[t].sum(), 1.0, rtol=1e-6)
 
 
+def test_group_ties_keep_the_lower_group():
+    # groups 1 and 3 share the largest maximum; with one group kept it is group 1
+    E, G = 16, 4
+    l = np.full((2, E), -1.0, np.float32)
+    l[:, 4:8] = [0.5, 2.0, 0.1, 0.2]      # group 1
+    l[:, 12:16] = [2.0, 1.5, 1.4, 1.3]    # group 3: same maximum, better runners-up
+    idx, _ = oracle.router_topk(l, 2, score_fn="softmax", n_group=G, topk_group=1)
+    np.testing.assert_array_equal(idx, [[5, 4], [5, 4]])
+    idx, _ = oracle.router_topk(l, 3, score_fn="sigmoid", n_group=G, topk_group=2)
+    np.testing.assert_array_equal(idx, [[5, 12, 13], [5, 12, 13]])
+
+
 def test_brute_force_small_group_limited():
     # every choice of groups: the chosen set maximises the sum of logits among
     # sets drawn from the best topk_group groups (by group maximum)

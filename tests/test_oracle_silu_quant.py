@@ -88,9 +88,11 @@ def test_quantised_activation_properties():
             assert np.all(np.abs(deq - blk) <= half * (1 + 1e-6) + np.abs(blk) * 2.0 ** -23)
 
 
-def test_column_major_scales_are_the_transpose():
+@pytest.mark.parametrize("in_use", [33, 20])
+def test_column_major_scales_are_the_transpose(in_use):
+    # the column-major stride is the row capacity, whatever the rows in use
     gu, src = _problem(33, 384, 4)
-    a1, s1 = oracle.silu_quant(gu, src, rows_in_use=33)
-    a2, s2 = oracle.silu_quant(gu, src, rows_in_use=33, col_major=True)
+    a1, s1 = oracle.silu_quant(gu, src, rows_in_use=in_use, fill=0)
+    a2, s2 = oracle.silu_quant(gu, src, rows_in_use=in_use, col_major=True, fill=0)
     np.testing.assert_array_equal(a1, a2)
     np.testing.assert_array_equal(s1.T, s2)
