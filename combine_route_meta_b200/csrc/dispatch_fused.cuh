@@ -188,26 +188,29 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct(FusedArgs
     const int64_t S = (int64_t)a.T * a.k;
 
     if (t == a.T) {
-        // metadata CTA: histogram, scan, offsets, unused rows
+        // metadata CTA: histogram, scan, offsets, and recv_src = -1 past the
+        // last segment (without padding there are no gaps between segments).
+        // It runs beside the token CTAs and is about as long, so it is kept lean.
         int32_t *hist = sm, *off = sm + a.E;
         for (int32_t e = threadIdx.x; e < a.E; e += nt)
             hist[e] = 0;
         __syncthreads();
-        for (int64_t base = 0; base < S; base += (int64_t)nt * kFusedLoadRounds) {
+        const int32_t S32 = (int32_t)S; // S <= kFusedMaxEntries
+        for (int32_t base = 0; base < S32; base += nt * kFusedLoadRounds) {
             int32_t ev[kFusedLoadRounds];
 #pragma unroll
             for (int r = 0; r < kFusedLoadRounds; ++r) {
-                const int64_t i = base + (int64_t)r * nt + threadIdx.x;
-                ev[r] = i < S ? __ldg(a.topk_idx + i) : -1;
+                const int32_t i = base + r * nt + (int32_t)threadIdx.x;
+                ev[r] = i < S32 ? __ldg(a.topk_idx + i) : 0;
             }
 #pragma unroll
             for (int r = 0; r < kFusedLoadRounds; ++r) {
-                const int64_t i = base + (int64_t)r * nt + threadIdx.x;
-                const int32_t e = ev[r];
-                if (i < S && (e < 0 || e >= a.E))
+                if (base + r * nt + (int32_t)threadIdx.x >= S32)
+                    break;
+                if ((uint32_t)ev[r] < (uint32_t)a.E)
+                    atomicAdd(&hist[ev[r]], 1);
+                else
                     raise_error(a.err, MOE_DEV_BAD_INDEX);
-                else if (i < S)
-                    atomicAdd(&hist[e], 1);
             }
         }
         __syncthreads();
@@ -219,8 +222,8 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct(FusedArgs
         if (threadIdx.x == 0)
             a.expert_offset[a.E] = off[a.E];
         for (int32_t r = threadIdx.x; r <= a.R; r += nt)
-            a.rank_offset[r] = off[(int64_t)r * (a.E / a.R)];
-        block_fill_unused(a.rows_cap, a.E, a.recv_src, hist, off, 0, 1);
+            a.rank_offset[r] = off[r * (a.E / a.R)];
+        block_fill_tail(a.rows_cap, a.E, a.recv_src, off, 0, 1);
         return;
     }
 
@@ -239,7 +242,7 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct(FusedArgs
 #pragma unroll
         for (int j = 0; j < kK; ++j) {
             const int32_t e = j < a.k ? __ldg(a.topk_idx + mine + j) : -1;
-            own[j] = (e >= 0 && e < a.E) ? e : -1;
+            own[j] = (uint32_t)e < (uint32_t)a.E ? e : -1;
         }
     }
     int32_t ev[kFusedLoadRounds];
@@ -284,7 +287,7 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct(FusedArgs
             const int32_t i = base + r * nt + (int32_t)threadIdx.x;
             if (__all_sync(kFullMask, i >= S32))
                 break; // later rounds start further out
-            const int32_t e = (ev[r] >= 0 && ev[r] < a.E) ? ev[r] : kNone;
+            const int32_t e = (uint32_t)ev[r] < (uint32_t)a.E ? ev[r] : kNone;
             const int32_t before = i - mine32; // entry i precedes (t, j) when before < j
 #pragma unroll
             for (int j = 0; j < kK; ++j) {

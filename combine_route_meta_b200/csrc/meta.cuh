@@ -107,15 +107,15 @@ __device__ __forceinline__ void block_count(const MetaArgs &a, int64_t begin, in
 // and ends with a barrier.
 __device__ void block_offsets(const int32_t *cnt, int32_t *off, int32_t E, int32_t pad128)
 {
+    // Each round scans blockDim.x counts: shuffle scan inside every warp, then
+    // every warp scans the warp totals itself (shuffles again, no serial walk).
     __shared__ int32_t warp_sums[32];
-    __shared__ int32_t carry;
-    if (threadIdx.x == 0)
-        carry = 0;
-    __syncthreads();
     const unsigned lane = lane_id(), warp = threadIdx.x / kWarp;
     const int nt = blockDim.x;
+    const int nwarps = nt / kWarp;
+    int32_t carry = 0; // identical in every thread
     for (int32_t base = 0; base < E; base += nt) {
-        int32_t e = base + threadIdx.x;
+        const int32_t e = base + threadIdx.x;
         int32_t v = 0;
         if (e < E) {
             v = cnt[e];
@@ -125,22 +125,27 @@ __device__ void block_offsets(const int32_t *cnt, int32_t *off, int32_t E, int32
         int32_t incl = v;
 #pragma unroll
         for (int d = 1; d < kWarp; d <<= 1) {
-            int32_t n = __shfl_up_sync(kFullMask, incl, d);
+            const int32_t n = __shfl_up_sync(kFullMask, incl, d);
             if (lane >= (unsigned)d)
                 incl += n;
         }
         if (lane == kWarp - 1)
             warp_sums[warp] = incl;
         __syncthreads();
-        int32_t before = carry;
-        for (unsigned w = 0; w < warp; ++w)
-            before += warp_sums[w];
+        const int32_t ws = (int)lane < nwarps ? warp_sums[lane] : 0;
+        int32_t wincl = ws;
+#pragma unroll
+        for (int d = 1; d < kWarp; d <<= 1) {
+            const int32_t n = __shfl_up_sync(kFullMask, wincl, d);
+            if (lane >= (unsigned)d)
+                wincl += n;
+        }
+        const int32_t before = __shfl_sync(kFullMask, wincl - ws, warp); // exclusive, this warp
+        const int32_t total = __shfl_sync(kFullMask, wincl, kWarp - 1);
         if (e < E)
-            off[e] = before + incl - v;
-        __syncthreads();
-        if (threadIdx.x == nt - 1)
-            carry = before + incl;
-        __syncthreads();
+            off[e] = carry + before + incl - v;
+        carry += total;
+        __syncthreads(); // warp_sums is rewritten by the next round
     }
     if (threadIdx.x == 0)
         off[E] = carry;
@@ -205,6 +210,17 @@ __device__ __forceinline__ void block_assign(const MetaArgs &a, int64_t begin, i
 // recv_src = -1 on rows that hold no entry: each expert's padding, and the rows
 // from expert_offset[E] to rows_cap.  Work is split over `nblk` blocks; inside
 // a block, one warp clears one expert's padding (at most 127 rows).
+// recv_src = -1 on the rows past the last segment, [off[E], rows_cap).
+__device__ __forceinline__ void block_fill_tail(int64_t rows_cap, int32_t E, int32_t *recv_src,
+                                                const int32_t *off, int blk, int nblk)
+{
+    for (int64_t r = (int64_t)off[E] + (int64_t)blk * blockDim.x + threadIdx.x; r < rows_cap;
+         r += (int64_t)nblk * blockDim.x)
+        recv_src[r] = -1;
+}
+
+// recv_src = -1 on every row no entry fills: the padding at the end of each
+// expert's segment and the rows past the last segment.
 __device__ __forceinline__ void block_fill_unused(int64_t rows_cap, int32_t E, int32_t *recv_src,
                                                   const int32_t *cnt, const int32_t *off, int blk,
                                                   int nblk)
@@ -217,9 +233,7 @@ __device__ __forceinline__ void block_fill_unused(int64_t rows_cap, int32_t E, i
         for (int64_t r = lo + lane; r < hi; r += kWarp)
             recv_src[r] = -1;
     }
-    for (int64_t r = (int64_t)off[E] + (int64_t)blk * blockDim.x + threadIdx.x; r < rows_cap;
-         r += (int64_t)nblk * blockDim.x)
-        recv_src[r] = -1;
+    block_fill_tail(rows_cap, E, recv_src, off, blk, nblk);
 }
 
 // Writes expert_count, expert_offset and rank_offset from shared cnt/off.
