@@ -287,11 +287,13 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct(FusedArgs
             const int32_t i = base + r * nt + (int32_t)threadIdx.x;
             if (__all_sync(kFullMask, i >= S32))
                 break; // later rounds start further out
-            const int32_t e = (uint32_t)ev[r] < (uint32_t)a.E ? ev[r] : kNone;
+            // Compared as unsigned, an id outside [0, E) is above every valid own
+            // id, so bad ids count in neither term without a separate check.
+            const uint32_t e = (uint32_t)ev[r];
             const int32_t before = i - mine32; // entry i precedes (t, j) when before < j
 #pragma unroll
             for (int j = 0; j < kK; ++j) {
-                const int32_t o = kOwnInRegs ? own[kOwnInRegs ? j : 0] : s_own[j];
+                const uint32_t o = (uint32_t)(kOwnInRegs ? own[kOwnInRegs ? j : 0] : s_own[j]);
                 cnt[j] += e < o ? 1u : 0u;
                 cnt[j] += (e == o && before < j) ? 0x10000u : 0u;
             }

@@ -13,6 +13,7 @@
 #include "combine_partial.cuh"
 #include "common.cuh"
 #include "dispatch_fused.cuh"
+#include "dispatch_multi.cuh"
 #include "meta.cuh"
 #include "router.cuh"
 #include "scatter.cuh"
@@ -262,6 +263,29 @@ cudaError_t launch_small(bool fp8, int per, int32_t T, int sms, cudaStream_t s, 
     }
     const unsigned block = (unsigned)((chunks + chosen - 1) / chosen * kWarp);
     return launch(small_kernel(fp8, pad, big_k, chosen), grid, block, smem, s, f);
+}
+
+// The mid-size one-launch dispatch applies past the one-token-per-CTA kernels
+// up to kMultiMaxEntries entries, for fp8 payloads and for bf16 rows too narrow
+// for the bulk scatter (wider bf16 rows keep the bulk stores, whose write
+// stream is worth more than the metadata launches at these sizes).
+bool use_multi(const moe_config *c, int32_t T)
+{
+    const int64_t S = (int64_t)T * c->k;
+    const bool fp8 = c->flags & MOE_FP8;
+    return S > kFusedMaxEntries && S <= kMultiMaxEntries && (fp8 || !use_bulk_scatter(c->H, false));
+}
+
+cudaError_t launch_multi(bool fp8, int32_t T, int sms, cudaStream_t s, const FusedArgs &f)
+{
+    // one CTA per SM at most (one wave), each owning a contiguous run of tokens
+    void (*k)(FusedArgs, int32_t) = fp8 ? dispatch_multi<true> : dispatch_multi<false>;
+    const int32_t G = T < sms ? T : sms;
+    const int32_t n_ent = (T + G - 1) / G * f.k;
+    const size_t smem = multi_smem(f.E, n_ent);
+    if (cached_per_sm((const void *)k, kMultiThreads, smem) == 0)
+        return cudaErrorInvalidConfiguration;
+    return launch(k, (unsigned)G, (unsigned)kMultiThreads, smem, s, f, n_ent);
 }
 
 size_t workspace_bytes(const moe_config *c, int32_t T)
@@ -607,6 +631,27 @@ int run_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
         f.err = dev_err;
         const cudaError_t e = launch_small(fp8, per, T, dev->sms, s, f);
         if ((st = launched(e)) != MOE_OK)
+            return st;
+    } else if (use_multi(cfg, T)) {
+        FusedArgs f;
+        f.x = static_cast<const uint16_t *>(x);
+        f.topk_idx = topk_idx;
+        f.T = T;
+        f.H = cfg->H;
+        f.k = cfg->k;
+        f.E = cfg->E;
+        f.R = cfg->R;
+        f.pad128 = (cfg->flags & MOE_PAD128) ? 1 : 0;
+        f.rows_cap = out->rows_cap;
+        f.recv_x = out->recv_x;
+        f.recv_scale = out->recv_scale;
+        f.expert_count = out->expert_count;
+        f.expert_offset = out->expert_offset;
+        f.rank_offset = out->rank_offset;
+        f.recv_src = out->recv_src;
+        f.slot = slot;
+        f.err = dev_err;
+        if ((st = launched(launch_multi(fp8, T, dev->sms, s, f))) != MOE_OK)
             return st;
     } else {
         if ((st = launch_layout(cfg, T, topk_idx, out, slot, workspace, dev_err, s)) != MOE_OK ||

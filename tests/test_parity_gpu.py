@@ -175,7 +175,10 @@ CASES = [
     (149, 7168, 256, 8, 8, True, True, True),
     (256, 7168, 256, 8, 8, True, False, True),
     (170, 4096, 128, 8, 12, True, False, False), # k > 8 own ids from shared memory, duplicates
-    # one-CTA metadata + scatter: k > 16, or 2048 < S <= 4096
+    # past the one-token-per-CTA kernels: the one-launch mid-size kernel for fp8 or
+    # narrow bf16 rows with S <= 16384, else metadata kernels + scatter
+    (2048, 256, 64, 8, 8, True, True, True),     # S = 16384: the largest mid-size batch
+    (2049, 256, 64, 8, 8, True, True, True),     # S = 16392: tiled metadata + fp8 scatter
     (10, 128, 8, 2, 20, False, False, False),
     (600, 1032, 16, 4, 5, False, True, False),   # ragged last 512-column chunk (8 columns)
     (300, 1152, 8, 8, 8, True, True, True),      # 9 scales per row: no 16-byte scale stores
@@ -210,9 +213,12 @@ def test_empty_batch(fp8, pad128):
     assert np.all(g["recv_src"] == -1)
 
 
-def test_every_token_to_one_expert():
-    # the hot bin: all entries on expert 3, which the tiled path must still order exactly
-    T, k = 3000, 2
+@pytest.mark.parametrize("T", [3000, 9000], ids=["mid_size", "tiled"])
+def test_every_token_to_one_expert(T):
+    # the hot bin: every j = 0 entry on expert 3 and every j = 1 entry on expert 5,
+    # which both the mid-size kernel (S = 6000) and the tiled metadata (S = 18000)
+    # must still order exactly
+    k = 2
     x, _, w = random_problem(41, T, 128, 8, k)
     idx = np.full((T, k), 3, np.int32)
     idx[:, 1] = 5
@@ -420,6 +426,33 @@ def test_layout_then_payload_equals_dispatch(T, H, E, k, fp8, pad128):
     a, b = dispatch_host(buf), dispatch_host(ref)
     for key in a:
         np.testing.assert_array_equal(a[key], b[key], err_msg=key)
+
+
+@pytest.mark.parametrize("T,H,E,R,k,fp8,pad128", [
+    (300, 1152, 8, 8, 8, True, True),      # S = 2400: one-CTA layout
+    (2048, 64, 512, 8, 2, False, True),    # S = 4096: the largest one-CTA layout
+    (2049, 64, 512, 8, 2, False, True),    # S = 4098: the smallest tiled layout
+    (5000, 128, 256, 32, 8, True, False),  # tiled, several tiles
+])
+def test_layout_path_matches_oracle(T, H, E, R, k, fp8, pad128):
+    # moe_dispatch takes the one-launch kernel at these sizes; the separate
+    # layout and payload calls keep the one-CTA and tiled metadata kernels, which
+    # are compared with the oracle here
+    x, idx, w = random_problem(T * 3 + H, T, H, E, k, distinct=E >= k)
+    if T == 5000:
+        idx[: T // 2, 0] = 7  # a hot expert across many tiles
+    cfg = moe.make_config(H, k, E, R, fp8, pad128)
+    buf = moe.Buffers(cfg, T, "cuda")
+    buf.recv_x.view(torch.uint8).fill_(POISON)
+    if buf.recv_scale is not None:
+        buf.recv_scale.view(torch.uint8).fill_(POISON)
+    moe.check()
+    moe.dispatch_layout_into(buf, to_dev(idx))
+    moe.dispatch_payload_into(buf, bf16_to_dev(x))
+    assert moe.check() == 0
+    o = oracle.dispatch(x, idx, E=E, R=R, fp8=fp8, pad128=pad128, rows_cap=buf.rows_cap,
+                        recv_fill=POISON)
+    assert_dispatch_equal(dispatch_host(buf), o)
 
 
 @pytest.mark.parametrize("H,fp8", [(256, False), (2048, False), (512, True)])
