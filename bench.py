@@ -249,7 +249,7 @@ def graph_kernels(g):
 
 
 def short_kernel_name(mangled):
-    for k in ("dispatch_fused", "dispatch_direct", "scatter_bulk_bf16", "scatter_rows", "combine_rows",
+    for k in ("dispatch_fused", "dispatch_direct", "dispatch_multi", "scatter_bulk_bf16", "scatter_rows", "combine_rows",
               "meta_single_block", "meta_tile_count", "meta_tile_scan", "meta_tile_assign"):
         if k in mangled:
             return k
@@ -581,7 +581,7 @@ def run_op(args, peak, peak_kind):
     gbs = nbytes / (us * 1e-6) / 1e9
     op_kernels = {"rank_partial": ["combine_partial_send", "combine_partial_recv"],
                   "silu_quant": ["silu_quant_rows"], "router": ["router_topk"],
-                  "route_dispatch": ["router_topk", "dispatch_direct", "dispatch_fused",
+                  "route_dispatch": ["router_topk", "dispatch_direct", "dispatch_fused", "dispatch_multi",
                                      "scatter_rows", "scatter_bulk_bf16"]}[args.op]
     extra["traffic"] = {k: recorded_traffic(k, w.name) for k in op_kernels}
     line = {"op": args.op, "workload": w.name, "us": round(us, 3), "algorithmic_bytes": nbytes,

@@ -9,19 +9,19 @@
 // fixed here as (token, k) ascending, which makes slot assignment a stable
 // counting sort of the S = T*k routing entries by expert id.
 //
-// GPU design.  Entries are processed in rounds of one entry per thread.  In a
-// round, lanes of a warp holding the same expert find each other with
-// __match_any_sync: the lowest such lane does one shared-memory update for the
-// whole group (so a skewed routing where most tokens pick one expert does not
-// serialise on one counter), and a lane's rank inside the group is the
-// population count of the group's lanes below it.  A lane's slot is then
+// GPU design.  Entries are processed in rounds of one entry per thread.  The
+// counts are plain shared-memory atomics.  For the slots, lanes of a warp
+// holding the same expert find each other with __match_any_sync: the lowest
+// such lane does one shared-memory update for the whole group, and a lane's
+// rank inside the group is the population count of the group's lanes below
+// it.  A lane's slot is then
 //   cursor[e]                          (rows handed out to e by earlier rounds)
 // + sum over lower warps of their group sizes for e   (this round)
 // + rank inside its own warp's group.
 // That is exactly the stable order, with no sort and no global atomics.
 //
-// Launch shapes (small decode batches take the fused kernel in
-// dispatch_fused.cuh instead):
+// Launch shapes (moe_dispatch takes the one-launch kernels of dispatch_fused.cuh
+// and dispatch_multi.cuh where they apply; moe_dispatch_layout always uses these):
 //  - S <= kSingleBlockEntries: one CTA does counts, scan and slots in shared
 //    memory (one launch, no scratch);
 //  - larger batches: tiles of kTileEntries entries.  (1) each CTA counts its
@@ -83,22 +83,20 @@ __device__ __forceinline__ void load_entries(const MetaArgs &a, int64_t begin, i
 }
 
 // Adds the entries [begin, end) into hist[E] (shared memory);
-// end - begin <= kRounds * kMetaThreads.
+// end - begin <= kRounds * kMetaThreads.  Plain shared-memory atomics: equal
+// ids in a warp serialise only as far as they repeat, and grouping them first
+// with __match_any_sync cost more on sm_100 than it saved, even for a Zipf-hot
+// expert.
 template <int kRounds>
 __device__ __forceinline__ void block_count(const MetaArgs &a, int64_t begin, int64_t end,
                                             int32_t *hist)
 {
     int32_t e[kRounds];
     load_entries<kRounds>(a, begin, end, true, e);
-    const unsigned lane = lane_id();
 #pragma unroll
-    for (int r = 0; r < kRounds; ++r) {
-        if (begin + (int64_t)r * kMetaThreads >= end)
-            break;
-        const unsigned peers = __match_any_sync(kFullMask, e[r]);
-        if (e[r] >= 0 && lane == (unsigned)(__ffs(peers) - 1))
-            atomicAdd(&hist[e[r]], __popc(peers));
-    }
+    for (int r = 0; r < kRounds; ++r)
+        if (e[r] >= 0)
+            atomicAdd(&hist[e[r]], 1);
 }
 
 // Exclusive scan of the (optionally 128-padded) counts in shared memory:
