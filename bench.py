@@ -249,8 +249,9 @@ def graph_kernels(g):
 
 
 def short_kernel_name(mangled):
-    for k in ("dispatch_fused", "dispatch_direct", "dispatch_multi", "scatter_bulk_bf16", "scatter_rows", "combine_rows",
-              "meta_single_block", "meta_tile_count", "meta_tile_scan", "meta_tile_assign"):
+    for k in ("dispatch_fused", "dispatch_direct", "dispatch_multi", "scatter_bulk_bf16",
+              "scatter_rows", "combine_rows", "meta_single_block", "meta_tile_count",
+              "meta_tile_scan", "meta_tile_assign"):
         if k in mangled:
             return k
     return mangled
