@@ -269,11 +269,16 @@ cudaError_t launch_small(bool fp8, int per, int32_t T, int sms, cudaStream_t s, 
 // up to kMultiMaxEntries entries, for fp8 payloads and for bf16 rows too narrow
 // for the bulk scatter (wider bf16 rows keep the bulk stores, whose write
 // stream is worth more than the metadata launches at these sizes).
+// It also takes the small batches the one-token-per-CTA kernels do not: T at or
+// above the SM count (one CTA per SM owning a few tokens beats two waves or two
+// half-size CTAs per SM) and k > kFusedMaxK.
 bool use_multi(const moe_config *c, int32_t T)
 {
     const int64_t S = (int64_t)T * c->k;
     const bool fp8 = c->flags & MOE_FP8;
-    return S > kFusedMaxEntries && S <= kMultiMaxEntries && (fp8 || !use_bulk_scatter(c->H, false));
+    if (S <= kFusedMaxEntries)
+        return T > 0;
+    return S <= kMultiMaxEntries && (fp8 || !use_bulk_scatter(c->H, false));
 }
 
 cudaError_t launch_multi(bool fp8, int32_t T, int sms, cudaStream_t s, const FusedArgs &f)
@@ -610,7 +615,8 @@ int run_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
     const bool fp8 = cfg->flags & MOE_FP8;
 
     unsigned fused_block = 0;
-    if (const int per = fused_chunks(cfg, T, &fused_block)) {
+    const int per = T < dev->sms ? fused_chunks(cfg, T, &fused_block) : 0;
+    if (per != 0) {
         FusedArgs f;
         f.x = static_cast<const uint16_t *>(x);
         f.topk_idx = topk_idx;
