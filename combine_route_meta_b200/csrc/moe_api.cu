@@ -173,9 +173,9 @@ int64_t rows_capacity(const moe_config *c, int32_t T)
 
 bool use_single_block(int64_t S) { return S <= kSingleBlockEntries; }
 
-// Chunks per warp of the fused small-batch dispatch (1, 2 or 4), or 0 if the
-// fused kernel does not apply.  *threads receives its block size.
-int fused_chunks(const moe_config *c, int32_t T, unsigned *threads)
+// Chunks per warp of the one-token-per-CTA dispatch (1, 2 or 4: the fewest that
+// fit the row in one CTA), or 0 if those kernels do not apply.
+int fused_chunks(const moe_config *c, int32_t T)
 {
     const int64_t S = (int64_t)T * c->k;
     const int32_t chunks = (c->H + chunk_cols<kFusedLaneCols>() - 1) / chunk_cols<kFusedLaneCols>();
@@ -183,10 +183,8 @@ int fused_chunks(const moe_config *c, int32_t T, unsigned *threads)
         return 0;
     const int max_warps = kFusedMaxThreads / kWarp;
     for (int per = 1; per <= kFusedMaxChunks; per *= 2)
-        if (chunks <= max_warps * per) {
-            *threads = (unsigned)((chunks + per - 1) / per) * kWarp;
+        if (chunks <= max_warps * per)
             return per;
-        }
     return 0;
 }
 
@@ -239,30 +237,17 @@ int cached_per_sm(const void *fn, int block, size_t smem)
     return n;
 }
 
-// Launches the one-token-per-CTA dispatch.  Chunks per warp start at `per`
-// (the fewest that fit the row in one CTA) and grow while the grid would not
-// be resident in one wave: at T near or above the SM count, two CTAs of half
-// the warps per SM beat two waves of one.
-cudaError_t launch_small(bool fp8, int per, int32_t T, int sms, cudaStream_t s, const FusedArgs &f)
+// Launches the one-token-per-CTA dispatch with `per` chunks per warp (the
+// fewest that fit the row in one CTA).  It runs only for T below the SM count
+// (larger small batches take dispatch_multi), so its T (+1) CTAs of at most
+// 1024 threads are resident in one wave.
+cudaError_t launch_small(bool fp8, int per, int32_t T, cudaStream_t s, const FusedArgs &f)
 {
-    const size_t smem = fused_smem(f.E);
     const bool pad = f.pad128 != 0;
-    const bool big_k = f.k > 8;
     const unsigned grid = pad ? (unsigned)T : (unsigned)T + 1;
     const int32_t chunks = (f.H + chunk_cols<kFusedLaneCols>() - 1) / chunk_cols<kFusedLaneCols>();
-    int chosen = per;
-    for (int p = per; p <= kFusedMaxChunks; p *= 2) {
-        const int block = (chunks + p - 1) / p * kWarp;
-        const int n = cached_per_sm((const void *)small_kernel(fp8, pad, big_k, p), block, smem);
-        if (n == 0)
-            return cudaErrorInvalidConfiguration;
-        if ((int64_t)grid <= (int64_t)sms * n) {
-            chosen = p;
-            break;
-        }
-    }
-    const unsigned block = (unsigned)((chunks + chosen - 1) / chosen * kWarp);
-    return launch(small_kernel(fp8, pad, big_k, chosen), grid, block, smem, s, f);
+    const unsigned block = (unsigned)((chunks + per - 1) / per * kWarp);
+    return launch(small_kernel(fp8, pad, f.k > 8, per), grid, block, fused_smem(f.E), s, f);
 }
 
 // The mid-size one-launch dispatch applies past the one-token-per-CTA kernels
@@ -614,8 +599,7 @@ int run_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
     int st;
     const bool fp8 = cfg->flags & MOE_FP8;
 
-    unsigned fused_block = 0;
-    const int per = T < dev->sms ? fused_chunks(cfg, T, &fused_block) : 0;
+    const int per = T < dev->sms ? fused_chunks(cfg, T) : 0;
     if (per != 0) {
         FusedArgs f;
         f.x = static_cast<const uint16_t *>(x);
@@ -635,7 +619,7 @@ int run_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
         f.recv_src = out->recv_src;
         f.slot = slot;
         f.err = dev_err;
-        const cudaError_t e = launch_small(fp8, per, T, dev->sms, s, f);
+        const cudaError_t e = launch_small(fp8, per, T, s, f);
         if ((st = launched(e)) != MOE_OK)
             return st;
     } else if (use_multi(cfg, T)) {

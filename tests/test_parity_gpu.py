@@ -305,10 +305,13 @@ def test_runs_are_bitwise_deterministic():
     np.testing.assert_array_equal(outs[0][1], outs[1][1])
 
 
-def test_graph_capture_replays_the_same_result():
+@pytest.mark.parametrize("name,over", [("dsv3_decode", {}), ("sweep_1024", {}),
+                                       ("sweep_4096", {"H": 512})],
+                         ids=["one_token_per_cta", "mid_size", "tiled"])
+def test_graph_capture_replays_the_same_result(name, over):
     # no host read-back inside dispatch/combine: the pair can be captured and replayed
-    w, x, idx, wts = make_inputs("dsv3_decode")
-    cfg = moe.make_config(w.H, w.k, w.E, w.R, True, False)
+    w, x, idx, wts = make_inputs(name, **over)
+    cfg = moe.make_config(w.H, w.k, w.E, w.R, w.fp8, w.pad128)
     buf = moe.Buffers(cfg, w.T, "cuda")
     xd, idd, wd = bf16_to_dev(x), to_dev(idx), to_dev(wts)
     eo = bf16_to_dev(make_expert_out(w, buf.rows_cap))
@@ -328,13 +331,45 @@ def test_graph_capture_replays_the_same_result():
     y.zero_()
     g.replay()
     torch.cuda.synchronize()
-    o = oracle.dispatch(x, idx, E=w.E, R=w.R, fp8=True, rows_cap=buf.rows_cap)
+    o = oracle.dispatch(x, idx, E=w.E, R=w.R, fp8=w.fp8, pad128=w.pad128, rows_cap=buf.rows_cap)
     gd = dispatch_host(buf)
     np.testing.assert_array_equal(gd["slot"], o["slot"])
     valid = o["recv_src"] >= 0
     np.testing.assert_array_equal(gd["recv_x"][valid], o["recv_x"][valid])
     ref = oracle.combine(o["slot"], wts, bf16_from_dev(eo))
     assert_combine_close(bf16_from_dev(y), ref)
+    assert moe.check() == 0
+
+
+def test_graph_capture_of_router_then_dispatch():
+    # router + dispatch in one call, captured: the replay routes and dispatches afresh
+    T, E, R, k, H = 128, 256, 8, 8, 7168
+    rng = np.random.default_rng(17)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    x = f32_to_bf16_bits(rng.standard_normal((T, H)).astype(np.float32))
+    cfg = moe.make_config(H, k, E, R, True, False)
+    buf = moe.Buffers(cfg, T, "cuda")
+    ld, xd = to_dev(logits), bf16_to_dev(x)
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    wt = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        moe.route_dispatch_into(buf, xd, ld, idx, wt, score_fn="sigmoid", n_group=8, topk_group=4,
+                                stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        moe.route_dispatch_into(buf, xd, ld, idx, wt, score_fn="sigmoid", n_group=8, topk_group=4)
+    idx.fill_(-1)
+    buf.slot.fill_(-5)
+    g.replay()
+    torch.cuda.synchronize()
+    ref_idx, _ = oracle.router_topk(logits, k, score_fn="sigmoid", n_group=8, topk_group=4)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
+    o = oracle.dispatch(x, ref_idx, E=E, R=R, fp8=True, rows_cap=buf.rows_cap)
+    np.testing.assert_array_equal(buf.slot.cpu().numpy(), o["slot"])
     assert moe.check() == 0
 
 
