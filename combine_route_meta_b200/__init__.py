@@ -113,6 +113,14 @@ def _declare(lib):
                                        ctypes.POINTER(moe_dispatch_out), P, P, ctypes.c_size_t, P, P,
                                        ctypes.POINTER(moe_handle)]
     lib.moe_route_dispatch.restype = ctypes.c_int
+    lib.moe_ep_rows_capacity.argtypes, lib.moe_ep_rows_capacity.restype = [cfgp, i32], i64
+    lib.moe_ep_layout.argtypes = [cfgp, i32, i32, P, P, P, P, i64, P, P, P, P, P]
+    lib.moe_ep_layout.restype = ctypes.c_int
+    lib.moe_ep_dispatch_payload.argtypes = [cfgp, i32, P, P, P, ctypes.POINTER(P), ctypes.POINTER(P),
+                                            i64, P, P]
+    lib.moe_ep_dispatch_payload.restype = ctypes.c_int
+    lib.moe_ep_combine.argtypes = [cfgp, i32, P, P, P, ctypes.POINTER(P), i64, P, P, P]
+    lib.moe_ep_combine.restype = ctypes.c_int
     lib.moe_check.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
     lib.moe_check.restype = ctypes.c_int
     return lib
@@ -137,6 +145,10 @@ moe_combine_rank_partial = lib.moe_combine_rank_partial
 moe_silu_quant = lib.moe_silu_quant
 moe_router_topk = lib.moe_router_topk
 moe_route_dispatch = lib.moe_route_dispatch
+moe_ep_rows_capacity = lib.moe_ep_rows_capacity
+moe_ep_layout = lib.moe_ep_layout
+moe_ep_dispatch_payload = lib.moe_ep_dispatch_payload
+moe_ep_combine = lib.moe_ep_combine
 
 
 class MoeError(RuntimeError):
@@ -446,3 +458,62 @@ def route_dispatch(x: torch.Tensor, logits: torch.Tensor, k: int, num_experts: i
     handle = Handle(buf.handle_c, buf.slot, w)
     return (DispatchResult(buf.recv_x, buf.recv_scale, buf.expert_count, buf.expert_offset,
                            buf.rank_offset, buf.recv_src, handle), idx, w)
+
+
+# ---- expert parallelism across ranks (see the C header) ------------------------------
+
+def ep_rows_capacity(cfg: moe_config, T: int) -> int:
+    """Rows of one rank's receive buffer when every rank dispatches up to T tokens."""
+    n = lib.moe_ep_rows_capacity(ctypes.byref(cfg), T)
+    if n < 0:
+        raise MoeError(ERR_INVALID_ARG, "moe_ep_rows_capacity")
+    return int(n)
+
+
+def _ptr_table(bufs):
+    """A ctypes array of device pointers from tensors (or ints, or None)."""
+    if bufs is None:
+        return None
+    vals = [b if isinstance(b, int) else (None if b is None else b.data_ptr()) for b in bufs]
+    return (ctypes.c_void_p * len(vals))(*vals)
+
+
+def ep_layout_into(cfg: moe_config, rank: int, topk_idx: torch.Tensor, local_slot: torch.Tensor,
+                   local_offset: torch.Tensor, counts_all: torch.Tensor, rows_cap: int,
+                   dst_row: torch.Tensor, recv_count: torch.Tensor, recv_offset: torch.Tensor,
+                   err: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None) -> None:
+    """moe_ep_layout into preallocated int32 tensors."""
+    P = ctypes.c_void_p
+    err = error_word(topk_idx.device) if err is None else err
+    st = lib.moe_ep_layout(ctypes.byref(cfg), rank, topk_idx.shape[0], P(topk_idx.data_ptr()),
+                           P(local_slot.data_ptr()), P(local_offset.data_ptr()), P(counts_all.data_ptr()),
+                           rows_cap, P(dst_row.data_ptr()), P(recv_count.data_ptr()),
+                           P(recv_offset.data_ptr()), P(err.data_ptr()), P(_stream_ptr(stream)))
+    _ok(st, "moe_ep_layout")
+
+
+def ep_dispatch_payload_into(cfg: moe_config, x: torch.Tensor, topk_idx: torch.Tensor,
+                             dst_row: torch.Tensor, peer_recv_x, peer_recv_scale, rows_cap: int,
+                             err: Optional[torch.Tensor] = None,
+                             stream: Optional[torch.cuda.Stream] = None) -> None:
+    """moe_ep_dispatch_payload; the peer tables are W tensors or device addresses."""
+    P = ctypes.c_void_p
+    err = error_word(x.device) if err is None else err
+    st = lib.moe_ep_dispatch_payload(ctypes.byref(cfg), x.shape[0], P(x.data_ptr()),
+                                     P(topk_idx.data_ptr()), P(dst_row.data_ptr()),
+                                     _ptr_table(peer_recv_x), _ptr_table(peer_recv_scale), rows_cap,
+                                     P(err.data_ptr()), P(_stream_ptr(stream)))
+    _ok(st, "moe_ep_dispatch_payload")
+
+
+def ep_combine_into(cfg: moe_config, topk_idx: torch.Tensor, dst_row: torch.Tensor,
+                    topk_w: torch.Tensor, peer_expert_out, rows_cap: int, y: torch.Tensor,
+                    err: Optional[torch.Tensor] = None,
+                    stream: Optional[torch.cuda.Stream] = None) -> None:
+    """moe_ep_combine into y[T, H] (bf16)."""
+    P = ctypes.c_void_p
+    err = error_word(y.device) if err is None else err
+    st = lib.moe_ep_combine(ctypes.byref(cfg), topk_idx.shape[0], P(topk_idx.data_ptr()),
+                            P(dst_row.data_ptr()), P(topk_w.data_ptr()), _ptr_table(peer_expert_out),
+                            rows_cap, P(y.data_ptr()), P(err.data_ptr()), P(_stream_ptr(stream)))
+    _ok(st, "moe_ep_combine")

@@ -1,0 +1,270 @@
+// Expert parallelism across GPUs: every rank dispatches its own tokens straight
+// into the receive buffers of the ranks that host their experts, and gathers
+// the experts' output rows back for its own combine.
+//
+// "Enabling trillion-parameter models on AWS EFA", sections "Buffers de Envio e
+// Recebimento" and "Despacho e Combinação": the ranks first share their
+// per-expert counts; from them every sender knows, for each peer, the
+// contiguous range its rows take in that peer's receive buffer, so one
+// receive buffer per rank suffices and each sender writes its rows straight
+// into it.  Inside a node the writes are NVLink stores to peer-mapped memory
+// (section "MoE all-to-all sobre EFA").
+//
+// Layout.  W ranks; rank d hosts experts [d E_l, (d+1) E_l), E_l = E / W.  With
+// cnt[s][e] the number of rank s's entries routed to expert e (gathered from
+// all ranks), rank d's receive buffer holds, expert by expert, the rows of rank
+// 0, then rank 1, ..., each in (token, k) order; with MOE_PAD128 every expert's
+// segment is padded to a multiple of 128 rows.  The row of rank s's entry
+// (t, j) with expert e in rank d's buffer is therefore
+//   off_d(e) + sum_{s' < s} cnt[s'][e] + (its rank among s's entries with e),
+// off_d(e) = sum over d's experts e' < e of the (padded) totals over ranks.
+// That is the single-GPU layout of all ranks' batches concatenated in rank
+// order, rank d's part starting at its rank offset, so the single-GPU oracle
+// fixes it.  A rank's own rank among its entries is slot - offset[e] of its
+// local, unpadded, one-rank layout (moe_dispatch_layout with R = 1).
+//
+// Peer buffers are reached through a table of W base pointers (peer mappings
+// of the other GPUs' buffers, this rank's own at its index).  Stores and loads
+// are plain 16-byte accesses; nothing here uses TMA or multicast, so the same
+// kernels are correct on peer memory.  Ordering between ranks is the caller's:
+// a stream synchronisation and a barrier between a payload and the peers' reads.
+#pragma once
+
+#include "combine.cuh"
+#include "common.cuh"
+#include "meta.cuh"
+#include "scatter.cuh"
+
+namespace moe {
+
+constexpr int kEpMaxRanks = 64;
+constexpr int kEpThreads = 256;
+
+struct EpPeers {
+    void *p[kEpMaxRanks];
+};
+
+struct EpRowsArgs {
+    const int32_t *topk_idx;     // [T, k] this rank's routing
+    const int32_t *local_slot;   // [T, k] its one-rank unpadded layout
+    const int32_t *local_offset; // [E + 1] of that layout
+    const int32_t *counts_all;   // [W, E] every rank's per-expert counts
+    int32_t T, k, E, W, rank, pad128;
+    int64_t rows_cap; // rows of every rank's receive buffer
+    int32_t *dst_row;     // [T, k] row in the destination rank's buffer, -1 if dropped
+    int32_t *recv_count;  // [E_l] this rank's experts' totals over ranks
+    int32_t *recv_offset; // [E_l + 1] their offsets in this rank's buffer
+    int32_t *err;
+};
+
+// Shared memory: tot[E], base[E], goff[E + 1].
+inline size_t ep_rows_smem(int32_t E) { return sizeof(int32_t) * ((size_t)3 * E + 1); }
+
+__global__ void __launch_bounds__(kEpThreads) ep_rows(EpRowsArgs a)
+{
+    stream_order_begin();
+    extern __shared__ int32_t sm[];
+    const int32_t E = a.E, El = a.E / a.W;
+    int32_t *tot = sm, *base = sm + E, *goff = sm + 2 * E;
+    for (int32_t e = threadIdx.x; e < E; e += blockDim.x) {
+        int32_t t = 0, b = 0;
+        for (int32_t s = 0; s < a.W; ++s) {
+            const int32_t c = __ldg(a.counts_all + (int64_t)s * E + e);
+            t += c;
+            if (s < a.rank)
+                b += c;
+        }
+        tot[e] = t;
+        base[e] = b;
+    }
+    __syncthreads();
+    // offsets over all experts; an expert's offset in its rank's buffer is the
+    // difference from the offset of that rank's first expert
+    block_offsets(tot, goff, E, a.pad128);
+    for (int32_t e = threadIdx.x; e < E; e += blockDim.x)
+        base[e] += goff[e] - goff[e / El * El];
+    __syncthreads();
+    if (blockIdx.x == 0) {
+        const int32_t e0 = a.rank * El;
+        for (int32_t i = threadIdx.x; i < El; i += blockDim.x) {
+            a.recv_count[i] = tot[e0 + i];
+            a.recv_offset[i] = goff[e0 + i] - goff[e0];
+        }
+        if (threadIdx.x == 0)
+            a.recv_offset[El] = goff[e0 + El] - goff[e0];
+    }
+    const int64_t S = (int64_t)a.T * a.k;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < S;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int32_t e = __ldg(a.topk_idx + i);
+        const int32_t s = __ldg(a.local_slot + i);
+        int32_t row = -1;
+        if ((uint32_t)e < (uint32_t)E && s >= 0) {
+            const int64_t r = (int64_t)base[e] + (s - __ldg(a.local_offset + e));
+            if (r < a.rows_cap)
+                row = (int32_t)r;
+            else
+                raise_error(a.err, MOE_DEV_CAPACITY);
+        }
+        a.dst_row[i] = row;
+    }
+}
+
+struct EpPayloadArgs {
+    const uint16_t *x;
+    const int32_t *topk_idx, *dst_row;
+    int32_t T, H, k, E, W;
+    int64_t rows_cap;
+    EpPeers recv_x;     // [W] receive buffers [rows_cap, H]
+    EpPeers recv_scale; // [W] fp8 scales [rows_cap, H/128]
+    int32_t *err;
+};
+
+// The destination row of entry j of a token (the same for the whole warp) and
+// its rank in d, or -1 when the entry is dropped; a row outside [-1, rows_cap)
+// is flagged and skipped, so no store or load leaves a buffer.
+__device__ __forceinline__ int64_t ep_entry(const int32_t *idx_t, const int32_t *row_t, int32_t j,
+                                            int32_t E, int32_t El, int64_t rows_cap, int32_t *err,
+                                            int32_t &d)
+{
+    const int32_t e = __ldg(idx_t + j);
+    const int32_t r = __ldg(row_t + j);
+    if (r == -1 || (uint32_t)e >= (uint32_t)E)
+        return -1;
+    if (r < 0 || r >= rows_cap) {
+        raise_error(err, MOE_DEV_BAD_SLOT);
+        return -1;
+    }
+    d = e / El;
+    return r;
+}
+
+// Warps walk (token, chunk) units as scatter_rows does; the k rows of a token
+// go to the buffers of the ranks hosting their experts.
+template <bool kFp8>
+__global__ void __launch_bounds__(kScatterThreads) ep_payload(EpPayloadArgs a)
+{
+    stream_order_begin();
+    constexpr int L = kScatterLaneCols;
+    const unsigned lane = lane_id();
+    const int32_t El = a.E / a.W;
+    const int64_t nwarps = (int64_t)gridDim.x * (kScatterThreads / kWarp);
+    const int32_t chunks = (a.H + chunk_cols<L>() - 1) / chunk_cols<L>();
+    const int64_t units = (int64_t)a.T * chunks;
+    const int32_t nb = a.H / 128;
+    for (int64_t u = (int64_t)blockIdx.x * (kScatterThreads / kWarp) + threadIdx.x / kWarp; u < units;
+         u += nwarps) {
+        const int32_t t = (int32_t)(u / chunks);
+        const int32_t c = (int32_t)(u % chunks);
+        LaneData<L> dl;
+        load_chunk<L, kFp8>(a.x + (int64_t)t * a.H, a.H, c, dl);
+        const int32_t *idx_t = a.topk_idx + (int64_t)t * a.k;
+        const int32_t *row_t = a.dst_row + (int64_t)t * a.k;
+        if constexpr (kFp8) {
+            LaneCodes<L> q;
+            quantise_lane<L>(dl, q.codes, q.scale);
+            const int32_t col = lane_col<L, true>(c, 0);
+            const bool active = col < a.H; // H % 128 == 0: whole blocks are in or out
+            for (int32_t j = 0; j < a.k; ++j) {
+                int32_t d = 0;
+                const int64_t r = ep_entry(idx_t, row_t, j, a.E, El, a.rows_cap, a.err, d);
+                if (r < 0)
+                    continue;
+                if (active) {
+                    uint8_t *dst = static_cast<uint8_t *>(a.recv_x.p[d]) + r * a.H + col;
+                    st_v4(dst, make_uint4(q.codes[0], q.codes[1], q.codes[2], q.codes[3]));
+                    if ((lane & (128 / L - 1)) == 0)
+                        static_cast<float *>(a.recv_scale.p[d])[r * nb + col / 128] = q.scale;
+                }
+            }
+        } else {
+            for (int32_t j = 0; j < a.k; ++j) {
+                int32_t d = 0;
+                const int64_t r = ep_entry(idx_t, row_t, j, a.E, El, a.rows_cap, a.err, d);
+                if (r < 0)
+                    continue;
+                uint16_t *dst = static_cast<uint16_t *>(a.recv_x.p[d]) + r * a.H;
+#pragma unroll
+                for (int i = 0; i < L / 8; ++i) {
+                    const int32_t col = lane_col<L, false>(c, i);
+                    if (col < a.H)
+                        st_v4(dst + col, dl.v[i]);
+                }
+            }
+        }
+    }
+}
+
+struct EpCombineArgs {
+    const int32_t *topk_idx, *dst_row;
+    const float *w;
+    int32_t T, H, k, E, W;
+    int32_t parts;
+    int64_t rows_cap;
+    EpPeers expert_out; // [W] expert outputs [rows_cap, H] bf16, receive layout
+    uint16_t *y;
+    int32_t *err;
+};
+
+// combine_rows with each entry's row read from the buffer of the rank that
+// hosts its expert: the same fp32 chain in ascending j, the same bf16 result.
+__global__ void __launch_bounds__(kCombineThreads) ep_combine(EpCombineArgs a)
+{
+    stream_order_begin();
+    const int32_t nvec = a.H / 8;
+    const int32_t El = a.E / a.W;
+    const int64_t units = (int64_t)a.T * a.parts;
+    for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
+        const int32_t t = (int32_t)(u / a.parts);
+        const int32_t v = (int32_t)(u % a.parts) * kCombineThreads + threadIdx.x;
+        if (v >= nvec)
+            continue;
+        const int32_t *idx_t = a.topk_idx + (int64_t)t * a.k;
+        const int32_t *row_t = a.dst_row + (int64_t)t * a.k;
+        const float *ws = a.w + (int64_t)t * a.k;
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            acc[i] = 0.0f;
+        for (int32_t j0 = 0; j0 < a.k; j0 += kCombineBatch) {
+            uint4 r[kCombineBatch];
+            bool use[kCombineBatch];
+#pragma unroll
+            for (int jj = 0; jj < kCombineBatch; ++jj) {
+                use[jj] = false;
+                r[jj] = make_uint4(0u, 0u, 0u, 0u);
+                if (j0 + jj < a.k) {
+                    int32_t d = 0;
+                    const int64_t row = ep_entry(idx_t, row_t, j0 + jj, a.E, El, a.rows_cap, a.err, d);
+                    if (row >= 0) {
+                        use[jj] = true;
+                        r[jj] = ld_stream_v4(static_cast<const uint16_t *>(a.expert_out.p[d]) +
+                                             row * a.H + (int64_t)v * 8);
+                    }
+                }
+            }
+#pragma unroll
+            for (int jj = 0; jj < kCombineBatch; ++jj) {
+                if (!use[jj])
+                    continue;
+                const float wj = __ldg(ws + j0 + jj);
+                acc[0] = fmaf(wj, bf16_lo(r[jj].x), acc[0]);
+                acc[1] = fmaf(wj, bf16_hi(r[jj].x), acc[1]);
+                acc[2] = fmaf(wj, bf16_lo(r[jj].y), acc[2]);
+                acc[3] = fmaf(wj, bf16_hi(r[jj].y), acc[3]);
+                acc[4] = fmaf(wj, bf16_lo(r[jj].z), acc[4]);
+                acc[5] = fmaf(wj, bf16_hi(r[jj].z), acc[5]);
+                acc[6] = fmaf(wj, bf16_lo(r[jj].w), acc[6]);
+                acc[7] = fmaf(wj, bf16_hi(r[jj].w), acc[7]);
+            }
+        }
+        uint4 out;
+        out.x = pack_bf16x2(acc[0], acc[1]);
+        out.y = pack_bf16x2(acc[2], acc[3]);
+        out.z = pack_bf16x2(acc[4], acc[5]);
+        out.w = pack_bf16x2(acc[6], acc[7]);
+        st_v4(a.y + (int64_t)t * a.H + (int64_t)v * 8, out);
+    }
+}
+
+} // namespace moe

@@ -14,6 +14,7 @@
 #include "common.cuh"
 #include "dispatch_fused.cuh"
 #include "dispatch_multi.cuh"
+#include "ep.cuh"
 #include "meta.cuh"
 #include "router.cuh"
 #include "scatter.cuh"
@@ -856,6 +857,166 @@ int moe_router_topk(int32_t T, int32_t E, int32_t k, const float *logits, int32_
         return st;
     return launch_router(T, E, k, logits, score_fn, n_group, topk_group, renormalize, topk_idx,
                          topk_w, dev, static_cast<cudaStream_t>(stream));
+}
+
+namespace {
+
+// Checks shared by the expert-parallel calls: cfg->R is the number of ranks.
+int check_ep(const moe_config *cfg, int32_t T, int64_t rows_cap)
+{
+    int st = check_config(cfg);
+    if (st != MOE_OK)
+        return st;
+    if (T < 0 || rows_cap < 0 || rows_cap > INT32_MAX)
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->R > kEpMaxRanks)
+        return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+int fill_peers(EpPeers *t, const void *const *peers, int32_t W, bool need)
+{
+    for (int32_t r = 0; r < kEpMaxRanks; ++r)
+        t->p[r] = nullptr;
+    if (!need)
+        return MOE_OK;
+    if (peers == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    for (int32_t r = 0; r < W; ++r) {
+        if (peers[r] == nullptr || !aligned16(peers[r]))
+            return MOE_ERR_INVALID_ARG;
+        t->p[r] = const_cast<void *>(peers[r]);
+    }
+    return MOE_OK;
+}
+
+} // namespace
+
+int64_t moe_ep_rows_capacity(const moe_config *cfg, int32_t T)
+{
+    if (check_config(cfg) != MOE_OK || T < 0 || cfg->R > kEpMaxRanks)
+        return -1;
+    const int64_t S = (int64_t)cfg->R * T * cfg->k; // every rank's entries to one rank
+    if (!(cfg->flags & MOE_PAD128))
+        return S;
+    const int64_t el = cfg->E / cfg->R;
+    const int64_t m = S < el ? S : el;
+    return (S + 127 * m) / 128 * 128;
+}
+
+int moe_ep_layout(const moe_config *cfg, int32_t rank, int32_t T, const int32_t *topk_idx,
+                  const int32_t *local_slot, const int32_t *local_offset, const int32_t *counts_all,
+                  int64_t rows_cap, int32_t *dst_row, int32_t *recv_count, int32_t *recv_offset,
+                  int32_t *dev_err, void *stream)
+{
+    int st = check_ep(cfg, T, rows_cap);
+    if (st != MOE_OK)
+        return st;
+    if (rank < 0 || rank >= cfg->R || counts_all == nullptr || recv_count == nullptr ||
+        recv_offset == nullptr || dev_err == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (topk_idx == nullptr || local_slot == nullptr || local_offset == nullptr ||
+                  dst_row == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    DeviceInfo *dev = nullptr;
+    if ((st = device_info(&dev)) != MOE_OK)
+        return st;
+    EpRowsArgs a;
+    a.topk_idx = topk_idx;
+    a.local_slot = local_slot;
+    a.local_offset = local_offset;
+    a.counts_all = counts_all;
+    a.T = T;
+    a.k = cfg->k;
+    a.E = cfg->E;
+    a.W = cfg->R;
+    a.rank = rank;
+    a.pad128 = (cfg->flags & MOE_PAD128) ? 1 : 0;
+    a.rows_cap = rows_cap;
+    a.dst_row = dst_row;
+    a.recv_count = recv_count;
+    a.recv_offset = recv_offset;
+    a.err = dev_err;
+    const int64_t S = (int64_t)T * cfg->k;
+    const unsigned grid = grid_for((S + kEpThreads - 1) / kEpThreads, dev->sms, 4);
+    return launched(launch(ep_rows, grid, kEpThreads, ep_rows_smem(cfg->E),
+                           static_cast<cudaStream_t>(stream), a));
+}
+
+int moe_ep_dispatch_payload(const moe_config *cfg, int32_t T, const void *x, const int32_t *topk_idx,
+                            const int32_t *dst_row, void *const *peer_recv_x,
+                            float *const *peer_recv_scale, int64_t rows_cap, int32_t *dev_err,
+                            void *stream)
+{
+    int st = check_ep(cfg, T, rows_cap);
+    if (st != MOE_OK)
+        return st;
+    const bool fp8 = cfg->flags & MOE_FP8;
+    if (dev_err == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0)
+        return MOE_OK;
+    if (x == nullptr || !aligned16(x) || topk_idx == nullptr || dst_row == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    EpPayloadArgs a;
+    if ((st = fill_peers(&a.recv_x, (const void *const *)peer_recv_x, cfg->R, true)) != MOE_OK ||
+        (st = fill_peers(&a.recv_scale, (const void *const *)peer_recv_scale, cfg->R, fp8)) != MOE_OK)
+        return st;
+    DeviceInfo *dev = nullptr;
+    if ((st = device_info(&dev)) != MOE_OK)
+        return st;
+    a.x = static_cast<const uint16_t *>(x);
+    a.topk_idx = topk_idx;
+    a.dst_row = dst_row;
+    a.T = T;
+    a.H = cfg->H;
+    a.k = cfg->k;
+    a.E = cfg->E;
+    a.W = cfg->R;
+    a.rows_cap = rows_cap;
+    a.err = dev_err;
+    const int64_t units = (int64_t)T * ((cfg->H + chunk_cols<kScatterLaneCols>() - 1) /
+                                        chunk_cols<kScatterLaneCols>());
+    const int64_t ctas = (units + kScatterThreads / kWarp - 1) / (kScatterThreads / kWarp);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const cudaError_t e = fp8 ? launch(ep_payload<true>, grid_for(ctas, dev->sms, 8), kScatterThreads, 0, s, a)
+                              : launch(ep_payload<false>, grid_for(ctas, dev->sms, 8), kScatterThreads, 0, s, a);
+    return launched(e);
+}
+
+int moe_ep_combine(const moe_config *cfg, int32_t T, const int32_t *topk_idx, const int32_t *dst_row,
+                   const float *topk_w, const void *const *peer_expert_out, int64_t rows_cap, void *y,
+                   int32_t *dev_err, void *stream)
+{
+    int st = check_ep(cfg, T, rows_cap);
+    if (st != MOE_OK)
+        return st;
+    if (dev_err == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0)
+        return MOE_OK;
+    if (topk_idx == nullptr || dst_row == nullptr || topk_w == nullptr || y == nullptr || !aligned16(y))
+        return MOE_ERR_INVALID_ARG;
+    EpCombineArgs a;
+    if ((st = fill_peers(&a.expert_out, peer_expert_out, cfg->R, true)) != MOE_OK)
+        return st;
+    DeviceInfo *dev = nullptr;
+    if ((st = device_info(&dev)) != MOE_OK)
+        return st;
+    a.topk_idx = topk_idx;
+    a.dst_row = dst_row;
+    a.w = topk_w;
+    a.T = T;
+    a.H = cfg->H;
+    a.k = cfg->k;
+    a.E = cfg->E;
+    a.W = cfg->R;
+    a.parts = (cfg->H / 8 + kCombineThreads - 1) / kCombineThreads;
+    a.rows_cap = rows_cap;
+    a.y = static_cast<uint16_t *>(y);
+    a.err = dev_err;
+    const unsigned grid = grid_for((int64_t)T * a.parts, dev->sms, 16);
+    return launched(launch(ep_combine, grid, kCombineThreads, 0, static_cast<cudaStream_t>(stream), a));
 }
 
 int moe_check(int32_t *dev_err, void *stream, int32_t *bits_out)

@@ -326,6 +326,64 @@ MOE_API int moe_route_dispatch(const moe_config *cfg, int32_t T, const void *x,
                                void *stream, moe_handle *handle);
 
 /*
+ * Expert parallelism across W GPUs ("Enabling trillion-parameter models on AWS
+ * EFA", sections "Buffers de Envio e Recebimento" and "Despacho e Combinação":
+ * the ranks share their per-expert counts first, and each sender then writes
+ * its rows into every peer's receive buffer at a range it computes itself).
+ * cfg->E is the global expert count and cfg->R the number of ranks W (at most
+ * 64, dividing E); rank d hosts experts [d*E/W, (d+1)*E/W).  Rank d's receive
+ * buffer holds, expert by expert, the rows from rank 0, then rank 1, ..., each
+ * in (token, k) order, each expert padded to 128 rows with MOE_PAD128: the
+ * single-GPU layout of all ranks' batches concatenated in rank order, from
+ * rank d's rank offset on.  Every rank calls, on its own stream:
+ *   1. moe_dispatch_layout with R = 1 and no padding on its own batch (its
+ *      counts, offsets and slots);
+ *   2. an all-gather of the E counts into counts_all[W, E] (the caller's
+ *      collective, e.g. NCCL);
+ *   3. moe_ep_layout, then moe_ep_dispatch_payload with the W receive buffers;
+ *   4. after a barrier that orders every rank's payload before the experts
+ *      read, and after the experts, moe_ep_combine with the W expert outputs.
+ * Buffer tables are host arrays of W device pointers (peer mappings; the
+ * rank's own buffer at its index), each 16-byte aligned, every buffer
+ * [rows_cap, H] (and [rows_cap, H/128] scales for fp8).  The kernels use plain
+ * loads and stores, so peer memory works as local memory does.
+ *
+ * moe_ep_rows_capacity: the rows one rank's buffer needs when every rank
+ * dispatches up to T tokens (all entries to one rank), or -1 on bad arguments.
+ *
+ * moe_ep_layout: from this rank's routing, its one-rank layout (local_slot
+ * [T,k], local_offset [E+1]) and counts_all [W,E] (device), writes dst_row
+ * [T,k] (the entry's row in the buffer of the rank hosting its expert; -1 for
+ * a bad id, and -1 with MOE_DEV_CAPACITY where the row is past rows_cap),
+ * recv_count [E/W] (this rank's experts' totals over all ranks) and recv_offset
+ * [E/W+1] (their offsets in this rank's buffer).
+ *
+ * moe_ep_dispatch_payload: copies (bf16) or quantises (MOE_FP8, as
+ * moe_dispatch does) x[t] into row dst_row[t,j] of the buffer of the rank that
+ * hosts topk_idx[t,j].  Rows outside [-1, rows_cap) set MOE_DEV_BAD_SLOT and are
+ * skipped.
+ *
+ * moe_ep_combine: y[t] = bf16(sum_j w[t,j] * row dst_row[t,j] of the expert
+ * output of the rank hosting topk_idx[t,j]), the fp32 chain of moe_combine.
+ *
+ * All return a status; argument errors enqueue nothing.
+ */
+MOE_API int64_t moe_ep_rows_capacity(const moe_config *cfg, int32_t T);
+MOE_API int moe_ep_layout(const moe_config *cfg, int32_t rank, int32_t T, const int32_t *topk_idx,
+                          const int32_t *local_slot, const int32_t *local_offset,
+                          const int32_t *counts_all, int64_t rows_cap, int32_t *dst_row,
+                          int32_t *recv_count, int32_t *recv_offset, int32_t *dev_err,
+                          void *stream);
+MOE_API int moe_ep_dispatch_payload(const moe_config *cfg, int32_t T, const void *x,
+                                    const int32_t *topk_idx, const int32_t *dst_row,
+                                    void *const *peer_recv_x, float *const *peer_recv_scale,
+                                    int64_t rows_cap, int32_t *dev_err, void *stream);
+MOE_API int moe_ep_combine(const moe_config *cfg, int32_t T, const int32_t *topk_idx,
+                           const int32_t *dst_row, const float *topk_w,
+                           const void *const *peer_expert_out, int64_t rows_cap, void *y,
+                           int32_t *dev_err, void *stream);
+
+/*
  * moe_dispatch without a workspace argument, for callers that cannot allocate
  * device memory (the pages have no counterpart; this is a deployment aid).
  *

@@ -114,6 +114,36 @@ def test_route_dispatch_checks_both_steps_before_launching():
     assert call(c=wide) == moe.ERR_UNSUPPORTED
 
 
+def test_expert_parallel_calls_check_their_arguments():
+    P = ctypes.c_void_p
+    cfg = moe.make_config(256, 2, 16, 4, fp8=False)                 # W = 4 ranks
+    assert moe.ep_rows_capacity(cfg, 10) == 4 * 10 * 2
+    pad = moe.make_config(256, 2, 16, 4, fp8=False, pad128=True)
+    assert moe.ep_rows_capacity(pad, 10) == (80 + 127 * 4) // 128 * 128   # 4 local experts
+    many = moe.make_config(256, 2, 128, 128, fp8=False)              # more ranks than supported
+    assert moe.moe_ep_rows_capacity(ctypes.byref(many), 10) == -1
+    args = [P(16)] * 4
+    # rank outside [0, W)
+    assert moe.moe_ep_layout(ctypes.byref(cfg), 4, 10, *args, 100, P(16), P(16), P(16), P(16),
+                             None) == moe.ERR_INVALID_ARG
+    assert moe.moe_ep_layout(ctypes.byref(many), 0, 10, *args, 100, P(16), P(16), P(16), P(16),
+                             None) == moe.ERR_UNSUPPORTED
+    table = (P * 4)(16, 32, None, 48)                                 # a missing peer buffer
+    assert moe.moe_ep_dispatch_payload(ctypes.byref(cfg), 10, P(16), P(16), P(16), table, None, 100,
+                                       P(16), None) == moe.ERR_INVALID_ARG
+    table = (P * 4)(16, 32, 40, 48)                                   # a misaligned one
+    assert moe.moe_ep_dispatch_payload(ctypes.byref(cfg), 10, P(16), P(16), P(16), table, None, 100,
+                                       P(16), None) == moe.ERR_INVALID_ARG
+    f8 = moe.make_config(256, 2, 16, 4, fp8=True)                     # fp8 without scale buffers
+    table = (P * 4)(16, 32, 64, 48)
+    assert moe.moe_ep_dispatch_payload(ctypes.byref(f8), 10, P(16), P(16), P(16), table, None, 100,
+                                       P(16), None) == moe.ERR_INVALID_ARG
+    assert moe.moe_ep_combine(ctypes.byref(cfg), 10, P(16), P(16), P(16), None, 100, P(16), P(16),
+                              None) == moe.ERR_INVALID_ARG
+    assert moe.moe_ep_combine(ctypes.byref(cfg), 10, P(16), P(16), P(16), table, -1, P(16), P(16),
+                              None) == moe.ERR_INVALID_ARG
+
+
 def test_combine_rejects_bad_arguments():
     h = moe.moe_handle(moe.make_config(256, 2, 8, 2, False), 16, 16, 16, 32)
     P = ctypes.c_void_p

@@ -71,3 +71,38 @@ def test_reference_arm_prints_from_rank_zero_only():
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["cores"] == 1
+
+
+def _counts_main(rank, world, port, out):
+    import datetime
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from combine_route_meta_b200.ep import exchange_counts
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        counts = torch.from_numpy(np.arange(8, dtype=np.int32) * (rank + 1))
+        got = exchange_counts(counts)
+        dist.barrier()
+        out[rank] = got.numpy().tolist()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_expert_parallel_count_exchange_two_gloo_ranks():
+    # the count exchange that precedes expert-parallel dispatch: every rank ends
+    # with every rank's per-expert counts, in rank order
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_counts_main, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    want = [[i * (r + 1) for i in range(8)] for r in range(2)]
+    assert out[0] == want and out[1] == want
