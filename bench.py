@@ -479,6 +479,7 @@ def partial_accuracy(moe, d, wts, b, w, dev, sample=64):
 
 def run_op(args, peak, peak_kind):
     """Times one next-row kernel on a workload's shapes; prints one JSON line."""
+    import dataclasses
     import math
     import torch
     import combine_route_meta_b200 as moe
@@ -535,6 +536,57 @@ def run_op(args, peak, peak_kind):
         fn = lambda b: (lambda: moe.route_dispatch_into(
             b["buf"], b["x"], b["l"], b["idx"], b["w"],
             score_fn="sigmoid" if w.routing == "sigmoid_topk" else "softmax", stream=stream))
+    elif args.op == "ep":
+        # W = the workload's R virtual ranks on this GPU, each with the workload's
+        # batch (its own routing seed); one launch = every rank's local layout,
+        # rows, payload and combine, the count exchange being each rank's
+        # counts written into its row of counts_all.  All buffers are local, so
+        # this times the kernels against HBM, not NVLink.
+        import ctypes
+        W = w.R
+        ranks = [make_inputs(dataclasses.replace(w, seed=w.seed + 101 * r)) for r in range(W)]
+        cfg = moe.make_config(w.H, w.k, w.E, W, w.fp8, w.pad128)
+        cfg1 = moe.make_config(w.H, w.k, w.E, 1, False, False)
+        cap = moe.ep_rows_capacity(cfg, w.T)
+        nws = moe.workspace_bytes(cfg1, w.T)
+        i32 = dict(dtype=torch.int32, device=dev)
+        fp8_dt = torch.float8_e4m3fn if w.fp8 else torch.bfloat16
+        set_bytes = W * cap * (w.H * (1 if w.fp8 else 2) + w.H * 2)
+        def make():
+            b = dict(counts=torch.empty((W, w.E), **i32), eo=[], recv_x=[], recv_sc=[], r=[])
+            for r in range(W):
+                _, xr, ir, wr = ranks[r]
+                b["recv_x"].append(torch.empty((cap, w.H), dtype=fp8_dt, device=dev))
+                b["recv_sc"].append(torch.empty((cap, w.H // 128), dtype=torch.float32, device=dev)
+                                    if w.fp8 else None)
+                b["eo"].append(bf16_dev(normal_bf16_rows(w.seed + r, 3, 0, cap, w.H)))
+                rr = dict(x=bf16_dev(xr), idx=torch.from_numpy(ir).to(dev), w=torch.from_numpy(wr).to(dev),
+                          off=torch.empty(w.E + 1, **i32), roff=torch.empty(2, **i32),
+                          src=torch.empty(S, **i32), slot=torch.empty((w.T, w.k), **i32),
+                          ws=torch.empty(max(nws, 1), dtype=torch.uint8, device=dev),
+                          dst=torch.empty((w.T, w.k), **i32), rc=torch.empty(w.E // W, **i32),
+                          ro=torch.empty(w.E // W + 1, **i32),
+                          y=torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev))
+                rr["out"] = moe.moe_dispatch_out(None, None, b["counts"][r].data_ptr(), rr["off"].data_ptr(),
+                                                 rr["roff"].data_ptr(), rr["src"].data_ptr(), S)
+                b["r"].append(rr)
+            return b
+        def ep_step(b):
+            P = ctypes.c_void_p
+            err = moe.error_word(dev)
+            for rr in b["r"]:
+                moe._ok(moe.moe_dispatch_layout(ctypes.byref(cfg1), w.T, P(rr["idx"].data_ptr()),
+                                                ctypes.byref(rr["out"]), P(rr["slot"].data_ptr()),
+                                                P(rr["ws"].data_ptr()), nws, P(err.data_ptr()),
+                                                P(stream.cuda_stream)), "layout")
+            for r, rr in enumerate(b["r"]):
+                moe.ep_layout_into(cfg, r, rr["idx"], rr["slot"], rr["off"], b["counts"], cap, rr["dst"],
+                                   rr["rc"], rr["ro"], err, stream)
+                moe.ep_dispatch_payload_into(cfg, rr["x"], rr["idx"], rr["dst"], b["recv_x"],
+                                             b["recv_sc"] if w.fp8 else None, cap, err, stream)
+            for rr in b["r"]:
+                moe.ep_combine_into(cfg, rr["idx"], rr["dst"], rr["w"], b["eo"], cap, rr["y"], err, stream)
+        fn = lambda b: (lambda: ep_step(b))
     else:
         raise SystemExit(f"unknown --op {args.op}")
     nsets = 1 if set_bytes >= 2 * l2 else min(64, math.ceil(2 * l2 / set_bytes) + 1)
@@ -576,12 +628,17 @@ def run_op(args, peak, peak_kind):
     elif args.op == "route_dispatch":
         nbytes = w.T * w.E * 4 + S * 8 + algorithmic_bytes(w.T, w.H, w.E, w.R, w.k, w.fp8)[0]
         extra = {}
+    elif args.op == "ep":
+        nbytes = sum(algorithmic_bytes(w.T * w.R, w.H, w.E, w.R, w.k, w.fp8))
+        extra = {"ranks": w.R, "tokens_per_rank": w.T, "kernels_per_launch": 4 * w.R,
+                 "note": "virtual ranks on one GPU: local buffers, HBM-bound, no NVLink"}
     else:
         nbytes = w.T * w.E * 4 + S * 8
         extra = {}
     gbs = nbytes / (us * 1e-6) / 1e9
     op_kernels = {"rank_partial": ["combine_partial_send", "combine_partial_recv"],
                   "silu_quant": ["silu_quant_rows"], "router": ["router_topk"],
+                  "ep": ["ep_rows", "ep_payload", "ep_combine"],
                   "route_dispatch": ["router_topk", "dispatch_direct", "dispatch_fused", "dispatch_multi",
                                      "scatter_rows", "scatter_bulk_bf16"]}[args.op]
     extra["traffic"] = {k: recorded_traffic(k, w.name) for k in op_kernels}
@@ -600,7 +657,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", default=None, choices=["rank_partial", "silu_quant", "router", "route_dispatch"],
+    ap.add_argument("--op", default=None, choices=["rank_partial", "silu_quant", "router", "route_dispatch",
+                                                   "ep"],
                     help="time one of the kernels next to the hot path instead of the step")
     args = ap.parse_args()
     if args.warmup < 3:
