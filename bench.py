@@ -552,6 +552,12 @@ def run_op(args, peak, peak_kind):
         i32 = dict(dtype=torch.int32, device=dev)
         fp8_dt = torch.float8_e4m3fn if w.fp8 else torch.bfloat16
         set_bytes = W * cap * (w.H * (1 if w.fp8 else 2) + w.H * 2)
+        # every rank's buffers hold the worst case (all entries to one rank), so
+        # many ranks with long batches would need far more memory than the GPU
+        # or the host generator can give; refuse those before allocating
+        if set_bytes > 8 << 30:
+            raise SystemExit(f"--op ep: {W} ranks x {cap} rows of worst-case buffers need "
+                             f"{set_bytes / 2**30:.0f} GiB; use a workload with fewer ranks or tokens")
         def make():
             b = dict(counts=torch.empty((W, w.E), **i32), eo=[], recv_x=[], recv_sc=[], r=[])
             for r in range(W):
