@@ -153,8 +153,9 @@ MOE_API int moe_dispatch_sizes_for(const moe_config *cfg, int32_t T, int64_t row
                            moe_dispatch_sizes *sizes);
 
 /*
- * Bytes of device scratch moe_dispatch needs for T tokens (0 for small
- * batches).  Returns 0 and sets nothing for an invalid cfg.
+ * Bytes of device scratch that moe_dispatch and moe_dispatch_layout require for
+ * T tokens (0 for small batches; where moe_dispatch takes a one-launch kernel it
+ * leaves the scratch untouched).  Returns 0 and sets nothing for an invalid cfg.
  */
 MOE_API size_t moe_workspace_bytes(const moe_config *cfg, int32_t T);
 
