@@ -167,3 +167,25 @@ def test_selftest_wait_rejects_bad_limits():
     assert moe.moe_selftest_bounded_wait(None, 1000, None) == moe.ERR_INVALID_ARG
     assert moe.moe_selftest_bounded_wait(P(16), 0, None) == moe.ERR_INVALID_ARG
     assert moe.moe_selftest_bounded_wait(P(16), 2_000_000_000, None) == moe.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("W,E,k,T", [(2, 4, 2, 3), (4, 8, 3, 2), (2, 2, 1, 5), (3, 9, 2, 2)])
+def test_ep_rows_capacity_is_the_worst_case(W, E, k, T):
+    # every way W ranks' entries (T tokens, k each) can land on one rank's E/W
+    # experts: the padded capacity is the most 128-row blocks they can fill,
+    # reached by spreading single entries over as many experts as possible
+    import itertools
+    import math
+    El = E // W
+    S = W * T * k
+    worst = 0
+    for n_experts in range(1, min(El, S) + 1):
+        # split S entries over n_experts non-empty experts; padding rounds each up
+        for parts in itertools.combinations_with_replacement(range(1, S + 1), n_experts):
+            if sum(parts) != S:
+                continue
+            worst = max(worst, sum(math.ceil(p / 128) * 128 for p in parts))
+    pad = moe.make_config(256, k, E, W, fp8=False, pad128=True)
+    assert moe.ep_rows_capacity(pad, T) == worst
+    plain = moe.make_config(256, k, E, W, fp8=False)
+    assert moe.ep_rows_capacity(plain, T) == S
