@@ -77,7 +77,7 @@ extern "C" {
 #define MOE_SCORE_SOFTMAX 0
 #define MOE_SCORE_SIGMOID 1
 
-/* Limits of this build. */
+/* Limits of this library. */
 #define MOE_MAX_EXPERTS 2048 /* E */
 #define MOE_MAX_TOPK 64      /* k */
 #define MOE_NO_ALLOC_SCRATCH_BYTES (1u << 20) /* fixed scratch of moe_dispatch_no_alloc */
