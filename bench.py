@@ -1,12 +1,19 @@
 """Benchmark of MoE dispatch + combine on B200 (one JSON line on stdout).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--per-config A,B|none] [--impl ours|reference] [--op OP]
 
 A step is one pass of the whole hot path -- routing metadata, dispatch payload
 (bf16 copy or fp8 block quantisation) and combine -- over one batch of
-synthetic inputs already resident in HBM.  Every step starts from a flushed L2
-(a 2x-L2 memset outside the timed events), and dispatch and combine replay as
-CUDA graphs, so the events time the GPU work and not Python.
+synthetic inputs already resident in HBM.  Steps replay as CUDA graphs that
+each hold a rotation of independent input/output sets, so that more than 2x L2
+of other data is touched between two uses of the same bytes (or one set alone
+is larger than 2x L2); there is no separate L2 flush.  The events bracket the
+replays on the launching stream, so they time the GPU work and not Python.
+
+The headline workload is the largest single-GPU batch (T=16384, H=7168, fp8
+dispatch with 128-row padding); `per_config` repeats the measurement for the
+other T >= 4096 configurations and for the DeepSeek-V3-shaped decode batch.
 
 `value` is the achieved HBM throughput of the step: the algorithmic bytes of
 dispatch + combine (x read once, k payload rows written per token, metadata;
@@ -29,7 +36,10 @@ import time
 import numpy as np
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-DEFAULT_WORKLOAD = "dsv3_decode"
+DEFAULT_WORKLOAD = "sweep_16384"
+PER_CONFIG = ("prefill_zipf", "sweep_4096", "dsv3_decode")
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e specification
+B200_L2_BYTES = 126 * 2**20  # nominal; the GPU arm sizes its rotation from the queried L2
 METRIC = "dispatch+combine µs and achieved HBM GB/s (% of B200 peak) per config"
 FALLBACK_HBM_GBS = 6650.0
 
@@ -257,9 +267,37 @@ def short_kernel_name(mangled):
     return mangled
 
 
-def run_gpu(args, rank, world):
-    import dataclasses
+def step_set_bytes(w, rows_cap):
+    """Bytes one step's input/output set occupies on the device."""
+    S = w.T * w.k
+    recv = rows_cap * w.H * (1 if w.fp8 else 2) + (rows_cap * (w.H // 128) * 4 if w.fp8 else 0)
+    eo = 0 if w.identity_experts else rows_cap * w.H * 2
+    return (w.T * w.H * 2 + S * 4 + S * 4 + eo + recv + rows_cap * 4 + S * 4 + w.T * w.H * 2)
+
+
+def rotating_sets(set_bytes, l2_bytes):
+    """Independent input/output sets to rotate through, so that more than 2x L2
+    of other sets' bytes is touched before a set is used again (1: one set is
+    already larger than 2x L2)."""
     import math
+    return 1 if set_bytes >= 2 * l2_bytes else min(64, math.ceil(2 * l2_bytes / set_bytes) + 1)
+
+
+def config_for(w, world, rows_cap):
+    """The `config` object of a JSON line; both arms print the same one."""
+    one_set = rotating_sets(step_set_bytes(w, rows_cap), B200_L2_BYTES) == 1
+    return {"workload": w.name, "T": w.T, "H": w.H, "E": w.E, "R": w.R, "k": w.k,
+            "payload": "fp8 e4m3 + fp32 scale per 128" if w.fp8 else "bf16",
+            "pad128": w.pad128, "combine": "bf16 out, fp32 accumulate",
+            "l2": ("inputs larger than 2x L2 every step (no flush needed)" if one_set else
+                   "rotating input sets: over 2x L2 of other sets touched between uses of a set"),
+            "graphs": "CUDA graphs of 8+ steps over the rotating sets, replayed back to back",
+            "parallelism": f"replicas x{world}"}
+
+
+def run_gpu(args, name, rank, world, with_e2e):
+    """Times K steps of one workload on this rank's GPU; returns the raw figures."""
+    import dataclasses
 
     import torch
     import combine_route_meta_b200 as moe
@@ -267,7 +305,7 @@ def run_gpu(args, rank, world):
 
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
-    w = dataclasses.replace(WORKLOADS[args.workload], seed=WORKLOADS[args.workload].seed + rank)
+    w = dataclasses.replace(WORKLOADS[name], seed=WORKLOADS[name].seed + rank)
     if w.identity_experts and w.fp8:
         raise SystemExit("identity experts need a bf16 dispatch")
     _, x, idx, wts = make_inputs(w)
@@ -282,10 +320,8 @@ def run_gpu(args, rank, world):
     # independent sets (inputs and outputs) that one step's data is evicted
     # before it comes round again.
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    recv_bytes = rows_cap * w.H * (1 if w.fp8 else 2) + (rows_cap * (w.H // 128) * 4 if w.fp8 else 0)
-    set_bytes = (x.nbytes + idx.nbytes + wts.nbytes + (0 if eo_host is None else eo_host.nbytes)
-                 + recv_bytes + rows_cap * 4 + idx.nbytes + w.T * w.H * 2)
-    nsets = 1 if set_bytes >= 2 * l2 else min(64, math.ceil(2 * l2 / set_bytes) + 1)
+    set_bytes = step_set_bytes(w, rows_cap)
+    nsets = rotating_sets(set_bytes, l2)
 
     class Set:
         pass
@@ -338,15 +374,16 @@ def run_gpu(args, rank, world):
     g_one = rotation(step_fn, 1)
     step_kernels = [short_kernel_name(k) for k in graph_kernels(g_one)]
     disp_kernels = [short_kernel_name(k) for k in graph_kernels(rotation(disp_fn, 1))]
+    del g_one
     launches_per_step = len(step_kernels)
     graph_cache = {}
 
     per_graph = max(nsets, 8)
 
-    def graphs_for(name, make, n):
+    def graphs_for(gname, make, n):
         """(full-rotation graph, remainder graph or None, rotations) covering n steps."""
         q, r = divmod(n, per_graph)
-        key = (name, r)
+        key = (gname, r)
         if key not in graph_cache:
             full = rotation(make, per_graph)
             full.instantiate()
@@ -358,21 +395,28 @@ def run_gpu(args, rank, world):
         full, rest = graph_cache[key]
         return full, rest, q
 
-    def run(name, make, n):
-        """Runs n steps of `make` back to back (rotating sets); device milliseconds."""
-        full, rest, q = graphs_for(name, make, n)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    def run(gname, make, n, per_replay=False):
+        """Runs n steps of `make` back to back (rotating sets).  Returns device
+        milliseconds, and with per_replay the milliseconds per step of each
+        full-rotation replay."""
+        full, rest, q = graphs_for(gname, make, n)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range((q if per_replay else 0) + 2)]
         with torch.cuda.stream(stream):
             # a sleeping kernel in front lets the host queue the replays ahead of the GPU
             torch.cuda._sleep(min(q + 1, 256) * 100_000)
-            e0.record(stream)
-            for _ in range(q):
+            ev[0].record(stream)
+            for i in range(q):
                 full.replay()
+                if per_replay:
+                    ev[i + 1].record(stream)
             if rest is not None:
                 rest.replay()
-            e1.record(stream)
-        e1.synchronize()
-        return e0.elapsed_time(e1)
+            ev[-1].record(stream)
+        ev[-1].synchronize()
+        total = ev[0].elapsed_time(ev[-1])
+        if not per_replay:
+            return total
+        return total, [ev[i].elapsed_time(ev[i + 1]) / per_graph for i in range(q)]
 
     # Warm-up: at least W steps, and on until the clock sampler reports (the GPU
     # is then under load when the timed region starts).
@@ -404,53 +448,123 @@ def run_gpu(args, rank, world):
     if dist is not None:
         total_ms = max_over_ranks(total_ms, dist, dev)
 
+    # Spread: the same K steps again with an event after every full-rotation
+    # replay (the events add a little time, so the headline is the pass above).
+    _, per_step_ms = run("step", step_fn, args.steps, per_replay=True)
+
     # Phase split, same protocol: K dispatches alone, K combines alone, and on the
     # multi-kernel dispatch path K payload kernels alone (moe_dispatch_payload on
     # the slots the last dispatch of each set left).
     disp_ms = run("disp", disp_fn, args.steps)
     comb_ms = run("comb", comb_fn, args.steps)
     pay_ms = run("pay", pay_fn, args.steps) if len(disp_kernels) > 1 else None
-
-    # End to end through the public API with host buffers: H2D of the step's
-    # inputs, dispatch, combine, D2H of y, every step.
-    st = sets[0]
-    pin = dict(pin_memory=True)
-    x_h = torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).pin_memory()
-    idx_h = torch.from_numpy(idx).pin_memory()
-    w_h = torch.from_numpy(wts).pin_memory()
-    eo_h = (None if eo_host is None else
-            torch.from_numpy(np.ascontiguousarray(eo_host).view(np.int16)).view(torch.bfloat16).pin_memory())
-    y_h = torch.empty((w.T, w.H), dtype=torch.bfloat16, **pin)
-    h2d = x_h.numel() * 2 + idx_h.numel() * 4 + w_h.numel() * 4 + (0 if eo_h is None else eo_h.numel() * 2)
-    d2h = y_h.numel() * 2
-    e2e_steps = max(3, min(args.steps, 20))
-    e2e_ms = []
     if dist is not None:
-        dist.barrier()  # every rank's copies share the node's host links while timed
-    for i in range(args.warmup + e2e_steps):
-        with torch.cuda.stream(stream):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            st.x.copy_(x_h, non_blocking=True)
-            st.idx.copy_(idx_h, non_blocking=True)
-            st.w.copy_(w_h, non_blocking=True)
-            if eo_h is not None:
-                st.eo.copy_(eo_h, non_blocking=True)
-            do_dispatch(st)
-            do_combine(st)
-            st.y_h = y_h.copy_(st.y, non_blocking=True)
-            e1.record(stream)
-        e1.synchronize()
-        if i >= args.warmup:
-            e2e_ms.append(e0.elapsed_time(e1))
-    e2e_med_ms = statistics.median(e2e_ms)
-    if dist is not None:
-        e2e_med_ms = max_over_ranks(e2e_med_ms, dist, dev)
+        disp_ms = max_over_ranks(disp_ms, dist, dev)
+        comb_ms = max_over_ranks(comb_ms, dist, dev)
+        if pay_ms is not None:
+            pay_ms = max_over_ranks(pay_ms, dist, dev)
+    graph_cache.clear()
 
-    return dict(w=w, total_ms=total_ms, disp_ms=disp_ms, comb_ms=comb_ms, pay_ms=pay_ms,
-                clocks=clocks, launches_per_step=launches_per_step, step_kernels=step_kernels,
-                disp_kernels=disp_kernels, e2e_med_ms=e2e_med_ms, h2d=h2d, d2h=d2h, nsets=nsets,
+    e2e = None
+    if with_e2e:
+        # End to end through the public API with host buffers: H2D of the step's
+        # inputs, dispatch, combine, D2H of y, every step.
+        st = sets[0]
+        pin = dict(pin_memory=True)
+        x_h = torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).pin_memory()
+        idx_h = torch.from_numpy(idx).pin_memory()
+        w_h = torch.from_numpy(wts).pin_memory()
+        eo_h = (None if eo_host is None else
+                torch.from_numpy(np.ascontiguousarray(eo_host).view(np.int16)).view(torch.bfloat16).pin_memory())
+        y_h = torch.empty((w.T, w.H), dtype=torch.bfloat16, **pin)
+        h2d = x_h.numel() * 2 + idx_h.numel() * 4 + w_h.numel() * 4 + (0 if eo_h is None else eo_h.numel() * 2)
+        d2h = y_h.numel() * 2
+        e2e_steps = max(3, min(args.steps, 20))
+        e2e_ms = []
+        if dist is not None:
+            dist.barrier()  # every rank's copies share the node's host links while timed
+        for i in range(args.warmup + e2e_steps):
+            with torch.cuda.stream(stream):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                st.x.copy_(x_h, non_blocking=True)
+                st.idx.copy_(idx_h, non_blocking=True)
+                st.w.copy_(w_h, non_blocking=True)
+                if eo_h is not None:
+                    st.eo.copy_(eo_h, non_blocking=True)
+                do_dispatch(st)
+                do_combine(st)
+                y_h.copy_(st.y, non_blocking=True)
+                e1.record(stream)
+            e1.synchronize()
+            if i >= args.warmup:
+                e2e_ms.append(e0.elapsed_time(e1))
+        e2e_med_ms = statistics.median(e2e_ms)
+        if dist is not None:
+            e2e_med_ms = max_over_ranks(e2e_med_ms, dist, dev)
+        if moe.check(stream) != 0:
+            raise RuntimeError("device error during the end-to-end steps")
+        e2e = dict(ms=e2e_med_ms, h2d=h2d, d2h=d2h)
+
+    sets.clear()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return dict(w=w, rows_cap=rows_cap, total_ms=total_ms, per_step_ms=per_step_ms, disp_ms=disp_ms,
+                comb_ms=comb_ms, pay_ms=pay_ms, clocks=clocks, launches_per_step=launches_per_step,
+                step_kernels=step_kernels, disp_kernels=disp_kernels, e2e=e2e, nsets=nsets,
                 set_bytes=set_bytes, l2=l2, per_graph=per_graph)
+
+
+def summarize(r, steps, world, peak, peak_kind):
+    """The per-workload figures of a JSON line: throughput, phase times, the
+    per-kernel rooflines and the clocks."""
+    w = r["w"]
+    db, cb = algorithmic_bytes(w.T, w.H, w.E, w.R, w.k, w.fp8)
+    step_bytes = db + cb
+    ms_per_step = r["total_ms"] / steps
+    value = job_throughput(step_bytes, world, ms_per_step)
+    disp_us = r["disp_ms"] / steps * 1e3
+    comb_us = r["comb_ms"] / steps * 1e3
+    # Per-kernel rooflines: the dispatch payload kernel (the fused kernel on the
+    # one-launch path) and the combine kernel, each timed alone over K launches.
+    S = w.T * w.k
+    kernels = []
+    if r["pay_ms"] is None:
+        kernels.append((r["disp_kernels"][0], db, disp_us))
+    else:
+        name = ([k for k in r["disp_kernels"] if k.startswith("scatter")] or ["payload"])[-1]
+        pay_bytes = (w.T * w.H * 2 + S * 4
+                     + (S * w.H + S * (w.H // 128) * 4 if w.fp8 else S * w.H * 2))
+        kernels.append((name, pay_bytes, r["pay_ms"] / steps * 1e3))
+    kernels.append(("combine_rows", combine_kernel_bytes(w.T, w.H, w.k), comb_us))
+    per_kernel = []
+    for name, nbytes, us in kernels:
+        gbs = nbytes / (us * 1e-6) / 1e9
+        per_kernel.append({"kernel": name, "us": round(us, 3), "algorithmic_bytes": nbytes,
+                           "achieved": round(gbs, 1), "frac": round(gbs / peak, 4),
+                           "traffic": recorded_traffic(name, w.name)})
+    dom = max(per_kernel, key=lambda k: k["us"])
+    roofline = {"bound": "hbm", "kernel": dom["kernel"], "achieved": dom["achieved"],
+                "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": dom["frac"],
+                "traffic": dom["traffic"], "algorithmic_bytes": dom["algorithmic_bytes"],
+                "kernels": per_kernel}
+    ps = sorted(r["per_step_ms"])
+    pct = lambda p: round(ps[min(len(ps) - 1, int(p * len(ps)))] * 1e3, 3) if ps else None
+    return {
+        "value": round(value, 1), "unit": "GB/s", "ms_per_step": round(ms_per_step, 5),
+        "dispatch_us": round(disp_us, 2), "combine_us": round(comb_us, 2),
+        "total_us": round(ms_per_step * 1e3, 2),
+        "pct_of_peak": round(100 * step_bytes / (ms_per_step * 1e-3) / 1e9 / peak, 2),
+        "pct_of_spec_peak": round(100 * step_bytes / (ms_per_step * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 2),
+        "bytes_per_step": {"dispatch": db, "combine": cb},
+        "step_us_spread": {"p10": pct(0.1), "p50": pct(0.5), "p90": pct(0.9), "replays": len(ps),
+                           "steps_per_replay": r["per_graph"]},
+        "roofline": roofline,
+        "kernels_per_step": r["step_kernels"],
+        "timing": {"sets": r["nsets"], "set_bytes": r["set_bytes"], "l2_bytes": r["l2"],
+                   "steps_per_graph": r["per_graph"]},
+        "clocks": r["clocks"],
+    }
 
 
 # ---- the rows next to the hot path: one kernel at a time ---------------------------
@@ -666,6 +780,10 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--per-config", default=None,
+                    help="comma-separated workloads measured after the headline one and reported "
+                         "under per_config (default: the other T >= 4096 configs and the decode "
+                         "config when the headline is the default; 'none' for none)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op", default=None, choices=["rank_partial", "silu_quant", "router", "route_dispatch",
@@ -678,8 +796,19 @@ def main():
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     from workloads import WORKLOADS
+    if args.workload not in WORKLOADS:
+        ap.error(f"unknown workload {args.workload}")
     w0 = WORKLOADS[args.workload]
     peak, peak_kind = measured_peak()
+    if args.per_config is None:
+        per_config = list(PER_CONFIG) if args.workload == DEFAULT_WORKLOAD else []
+    elif args.per_config.strip().lower() in ("", "none"):
+        per_config = []
+    else:
+        per_config = [p.strip() for p in args.per_config.split(",") if p.strip()]
+    for p in per_config:
+        if p not in WORKLOADS:
+            ap.error(f"unknown workload {p} in --per-config")
 
     if args.op is not None:
         run_op(args, peak, peak_kind)
@@ -689,19 +818,20 @@ def main():
         # The reference arm is the CPU oracle, timed on this host's cores (rank 0 only).
         if rank != 0:
             return
+        import oracle
         run = OracleRun(w0)
         per_step = [run.once() for _ in range(args.warmup + args.steps)][args.warmup:]
         total = sum(per_step)
         g = run.bytes * args.steps / total / 1e9
         ms = total / args.steps * 1e3
         desc = f"{run.desc}, {args.steps} timed runs"
+        cap = oracle.rows_capacity(w0.T, w0.k, w0.E, w0.pad128)
         line = {
             "impl": "reference", "metric": METRIC, "value": round(g, 3), "unit": "GB/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "T": w0.T, "H": w0.H, "E": w0.E, "R": w0.R,
-                       "k": w0.k, "payload": "fp8" if w0.fp8 else "bf16", "pad128": w0.pad128},
+            "config": config_for(w0, max(world, args.gpus), cap),
             "cpu_baseline": {"value": round(g, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": round(g, 3), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -714,66 +844,39 @@ def main():
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    r = run_gpu(args, rank, world)
+    r = run_gpu(args, args.workload, rank, world, with_e2e=True)
+    head = summarize(r, args.steps, world, peak, peak_kind)
     w = r["w"]
-    db, cb = algorithmic_bytes(w.T, w.H, w.E, w.R, w.k, w.fp8)
-    step_bytes = db + cb
-    ms_per_step = r["total_ms"] / args.steps
-    value = job_throughput(step_bytes, world, ms_per_step)
-
-    disp_us = r["disp_ms"] / args.steps * 1e3
-    comb_us = r["comb_ms"] / args.steps * 1e3
-    # Per-kernel rooflines: the dispatch payload kernel (the fused kernel on the
-    # one-launch path) and the combine kernel, each timed alone over K launches.
-    S = w.T * w.k
-    kernels = []
-    if r["pay_ms"] is None:
-        name = r["disp_kernels"][0]
-        kernels.append((name, db, disp_us, "dispatch_fused.cuh"))
-    else:
-        name = ([k for k in r["disp_kernels"] if k.startswith("scatter")] or ["payload"])[-1]
-        pay_bytes = (w.T * w.H * 2 + S * 4
-                     + (S * w.H + S * (w.H // 128) * 4 if w.fp8 else S * w.H * 2))
-        kernels.append((name, pay_bytes, r["pay_ms"] / args.steps * 1e3, "scatter.cuh"))
-    kernels.append(("combine_rows", combine_kernel_bytes(w.T, w.H, w.k), comb_us, "combine.cuh"))
-    per_kernel = []
-    for name, nbytes, us, src in kernels:
-        gbs = nbytes / (us * 1e-6) / 1e9
-        per_kernel.append({"kernel": name, "us": round(us, 3), "algorithmic_bytes": nbytes,
-                           "achieved": round(gbs, 1), "frac": round(gbs / peak, 4),
-                           "traffic": recorded_traffic(name, w.name)})
-    dom = max(per_kernel, key=lambda k: k["us"])
-    roofline = {"bound": "hbm", "kernel": dom["kernel"], "achieved": dom["achieved"],
-                "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": dom["frac"],
-                "traffic": dom["traffic"], "algorithmic_bytes": dom["algorithmic_bytes"],
-                "kernels": per_kernel}
-    e2e_ms = r["e2e_med_ms"]  # max over ranks of each rank's median
+    e2e = r["e2e"]
+    step_bytes = sum(head["bytes_per_step"].values())
+    launches = r["launches_per_step"] * args.steps * world
     line = {
-        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "metric": METRIC, "value": head["value"], "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": w.name, "T": w.T, "H": w.H, "E": w.E, "R": w.R, "k": w.k,
-                   "payload": "fp8 e4m3 + fp32 scale per 128" if w.fp8 else "bf16",
-                   "pad128": w.pad128, "combine": "bf16 out, fp32 accumulate",
-                   "l2": (f"{r['nsets']} rotating sets of {r['set_bytes'] / 1e6:.1f} MB "
-                          f"({r['nsets'] * r['set_bytes'] / 1e6:.0f} MB touched between uses of a "
-                          f"set; L2 {r['l2'] / 1e6:.0f} MB)"),
-                   "graphs": (f"CUDA graphs of {r['per_graph']} steps over the rotating sets, "
-                              "replayed back to back"),
-                   "parallelism": f"replicas x{world}"},
-        "dispatch_us": round(disp_us, 2), "combine_us": round(comb_us, 2),
-        "total_us": round(ms_per_step * 1e3, 2),
-        "pct_of_peak": round(100 * step_bytes / (ms_per_step * 1e-3) / 1e9 / peak, 2),
-        "bytes_per_step": {"dispatch": db, "combine": cb},
-        "roofline": roofline,
-        "e2e": {"value": round(job_throughput(step_bytes, world, e2e_ms), 3), "unit": "GB/s",
-                "h2d_bytes_per_step": r["h2d"] * world, "d2h_bytes_per_step": r["d2h"] * world,
-                "ms_per_step": round(e2e_ms, 4)},
-        "gpu_launches": r["launches_per_step"] * args.steps * world,
-        "kernels_per_step": r["step_kernels"],
-        "clocks": r["clocks"],
+        "config": config_for(w, world, r["rows_cap"]),
+        **{k: head[k] for k in ("dispatch_us", "combine_us", "total_us", "pct_of_peak",
+                                "pct_of_spec_peak", "bytes_per_step", "step_us_spread", "roofline")},
+        "e2e": {"value": round(job_throughput(step_bytes, world, e2e["ms"]), 3), "unit": "GB/s",
+                "h2d_bytes_per_step": e2e["h2d"] * world, "d2h_bytes_per_step": e2e["d2h"] * world,
+                "ms_per_step": round(e2e["ms"], 4)},
+        "kernels_per_step": head["kernels_per_step"],
+        "timing": head["timing"],
+        "clocks": head["clocks"],
     }
+    if per_config:
+        line["per_config"] = {}
+        for name in per_config:
+            rp = run_gpu(args, name, rank, world, with_e2e=False)
+            s = summarize(rp, args.steps, world, peak, peak_kind)
+            s["config"] = config_for(rp["w"], world, rp["rows_cap"])
+            line["per_config"][name] = s
+            launches += rp["launches_per_step"] * args.steps * world
+        # every timed pass above launched this library's kernels only
+    line["gpu_launches"] = launches
+    line["gpu_launches_note"] = ("kernel nodes of the captured step graph x K, over the headline "
+                                 "and per_config timed passes")
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         g, desc = time_oracle(w0)
         line["cpu_baseline"] = {"value": round(g, 4), "unit": "GB/s", "cores": 1,
