@@ -38,7 +38,7 @@ def build(force: bool = False) -> str:
                  or os.path.getmtime(_LIB) < os.path.getmtime(_SRC))
         if force or stale:
             tmp = _LIB + f".tmp{os.getpid()}"
-            subprocess.check_call(["gcc", *GCC_FLAGS, "-o", tmp, _SRC, "-lm"])
+            subprocess.check_call(["gcc", *GCC_FLAGS, "-o", tmp, _SRC, "-lquadmath", "-lm"])
             os.replace(tmp, _LIB)
     return _LIB
 
@@ -58,8 +58,10 @@ def _load():
         lib.oracle_combine.restype = None
         lib.oracle_combine_rank_partial.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P]
         lib.oracle_combine_rank_partial.restype = None
-        lib.oracle_silu_f32.argtypes = [ctypes.c_float]
-        lib.oracle_silu_f32.restype = ctypes.c_float
+        lib.oracle_silu_mul.argtypes = [ctypes.c_float, ctypes.c_float]
+        lib.oracle_silu_mul.restype = ctypes.c_float
+        lib.oracle_silu_mul_many.argtypes = [i64, P, P, P]
+        lib.oracle_silu_mul_many.restype = None
         lib.oracle_silu_quant.argtypes = [i64, i32, P, P, i64, P, P, i32]
         lib.oracle_silu_quant.restype = None
         lib.oracle_router_topk.argtypes = [i32, i32, i32, P, i32, i32, i32, i32, P, P]
@@ -196,9 +198,18 @@ def combine_rank_partial(topk_idx, slot, topk_w, expert_out_bf16, *, E: int, R: 
     return out
 
 
-def silu_f32(g: float) -> float:
-    """SiLU in binary32 as the oracle defines it (see moe_oracle.c)."""
-    return float(_load().oracle_silu_f32(float(np.float32(g))))
+def silu_mul(g: float, u: float = 1.0) -> float:
+    """The activation silu(g) * u: the binary32 value nearest the real one (see moe_oracle.c)."""
+    return float(_load().oracle_silu_mul(float(np.float32(g)), float(np.float32(u))))
+
+
+def silu_mul_bits(g_bf16, u_bf16) -> np.ndarray:
+    """silu_mul over arrays of bf16 bit patterns; float32 results of the same shape."""
+    g = _c(g_bf16, np.uint16)
+    u = _c(np.broadcast_to(u_bf16, g.shape), np.uint16)
+    out = np.empty(g.shape, np.float32)
+    _load().oracle_silu_mul_many(g.size, _ptr(g), _ptr(u), _ptr(out))
+    return out
 
 
 def silu_quant(gate_up_bf16, recv_src, rows_in_use: int, *, col_major: bool = False,

@@ -39,6 +39,7 @@
  *   - an all-zero 128-block gets scale 0 and all codes +0.
  */
 #include <math.h>
+#include <quadmath.h>
 #include <stdint.h>
 #include <string.h>
 #include <stdlib.h>
@@ -335,45 +336,37 @@ void oracle_combine_rank_partial(int32_t T, int32_t H, int32_t k, int32_t E, int
 }
 
 /*
- * e^x in binary32 for x in [-87, 88], by Cody-Waite argument reduction and a
- * degree-7 Taylor polynomial (Cody and Waite, "Software Manual for the
- * Elementary Functions", 1980): x = n*ln2 + r with n = rint(x*log2(e)) and
- * |r| <= ln2/2, r computed with ln2 split in a high part (exact products) and a
- * low part; e^r = sum_{i<=7} r^i/i! by Horner's rule with fused multiply-adds;
- * then scaled by 2^n.  Every step is one IEEE operation, so the value is a
- * fixed function of x.
+ * The activation of one (gate, up) pair: SiLU of the gate times the up value
+ * ("Lower latency and higher throughput with multi-node DeepSeek deployment",
+ * section "Quantização", where the SiLU kernel feeds the block quantiser).
+ * Its value is the binary32 number nearest to the real number
+ *
+ *     silu(g) * u = g * u / (1 + e^-g),
+ *
+ * ties to even, with g and u the exact values of the bf16 inputs; a zero result
+ * carries the sign of g * u, as an IEEE product does.  This is the plain
+ * definition, written out: the quotient is evaluated in binary128 (113-bit
+ * significands; g * u is exact there, e^-g comes from libquadmath's expq and
+ * overflows to +inf only where the result is a signed zero anyway) and
+ * converted to binary32 once.  The binary128 value is within a few units of
+ * 2^-112 (relative) of the real one, so the single conversion gives the
+ * nearest binary32 unless the real value lies closer than that to a point
+ * halfway between two binary32 numbers; silu(g) * u is transcendental for
+ * g, u != 0, so it is never exactly halfway, and the tests check the result
+ * against 50-digit decimal arithmetic.  Results beyond the binary32 range
+ * (|g * u| near 2^128) are out of contract.
  */
-static float exp_cody_waite(float x)
+float oracle_silu_mul(float g, float u)
 {
-    const float n = rintf(x * 1.44269504088896341f);
-    float r = fmaf(-n, 0.693145751953125f, x);
-    r = fmaf(-n, 1.42860682030941723212e-6f, r);
-    float p = 1.98412698412698413e-4f; /* 1/7! */
-    p = fmaf(p, r, 1.38888888888888889e-3f); /* 1/6! */
-    p = fmaf(p, r, 8.33333333333333333e-3f); /* 1/5! */
-    p = fmaf(p, r, 4.16666666666666667e-2f); /* 1/4! */
-    p = fmaf(p, r, 1.66666666666666667e-1f); /* 1/3! */
-    p = fmaf(p, r, 0.5f);
-    p = fmaf(p, r, 1.0f);
-    p = fmaf(p, r, 1.0f);
-    /* 2^n, n in [-126, 127], from its exponent bits */
-    const uint32_t bits = (uint32_t)((int32_t)n + 127) << 23;
-    float two_n;
-    memcpy(&two_n, &bits, sizeof two_n);
-    return p * two_n;
+    const __float128 G = g, U = u;
+    return (float)(G * U / ((__float128)1 + expq(-G)));
 }
 
-/* SiLU in binary32: g / (1 + e^-g).  Below g = -88 the result is -0 (the true
- * magnitude is under 5.3e-37); above g = 87, 1 + e^-g rounds to 1, so the
- * exponent argument is clamped at -87 without changing the result. */
-float oracle_silu_f32(float g)
+/* oracle_silu_mul over n pairs given as bf16 bits. */
+void oracle_silu_mul_many(int64_t n, const uint16_t *g, const uint16_t *u, float *out)
 {
-    if (g < -88.0f)
-        return -0.0f;
-    float x = -g;
-    if (x < -87.0f)
-        x = -87.0f;
-    return g / (1.0f + exp_cody_waite(x));
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = oracle_silu_mul(bf16_to_float(g[i]), bf16_to_float(u[i]));
 }
 
 /*
@@ -383,7 +376,7 @@ float oracle_silu_f32(float g)
  * largest magnitude of every 128-element block for its scale; it reads the
  * routing counts to know which rows are populated).
  *   gate_up [rows_cap, 2I] bf16: gate = columns [0, I), up = [I, 2I).
- *   a = silu(gate) * up (binary32), then per 128-block: scale = amax/448,
+ *   a = silu(gate) * up (oracle_silu_mul), then per 128-block: scale = amax/448,
  *   codes e4m3(a/scale) as in the dispatch quantiser.
  * Only rows r < rows_in_use with recv_src[r] >= 0 are written.  Scales are
  * row-major [rows_cap, I/128] or, with col_major, [I/128, rows_cap].
@@ -402,7 +395,7 @@ void oracle_silu_quant(int64_t rows_cap, int32_t I, const uint16_t *gate_up,
         const uint16_t *g = gate_up + r * 2 * (int64_t)I;
         const uint16_t *u = g + I;
         for (int32_t i = 0; i < I; ++i)
-            a[i] = oracle_silu_f32(bf16_to_float(g[i])) * bf16_to_float(u[i]);
+            a[i] = oracle_silu_mul(bf16_to_float(g[i]), bf16_to_float(u[i]));
         for (int32_t b = 0; b < nb; ++b) {
             float amax = 0.0f;
             for (int32_t i = 0; i < 128; ++i) {
