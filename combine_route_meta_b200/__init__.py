@@ -107,6 +107,8 @@ def _declare(lib):
     lib.moe_combine_rank_partial.restype = ctypes.c_int
     lib.moe_silu_quant.argtypes = [i64, i32, P, P, P, P, P, i32, P]
     lib.moe_silu_quant.restype = ctypes.c_int
+    lib.moe_silu_mul.argtypes = [i64, P, P, P, P, i32, P]
+    lib.moe_silu_mul.restype = ctypes.c_int
     lib.moe_router_topk.argtypes = [i32, i32, i32, P, i32, i32, i32, i32, P, P, P]
     lib.moe_router_topk.restype = ctypes.c_int
     lib.moe_route_dispatch.argtypes = [cfgp, i32, P, P, i32, i32, i32, i32, P, P,
@@ -143,6 +145,7 @@ moe_check = lib.moe_check
 moe_selftest_bounded_wait = lib.moe_selftest_bounded_wait
 moe_combine_rank_partial = lib.moe_combine_rank_partial
 moe_silu_quant = lib.moe_silu_quant
+moe_silu_mul = lib.moe_silu_mul
 moe_router_topk = lib.moe_router_topk
 moe_route_dispatch = lib.moe_route_dispatch
 moe_ep_rows_capacity = lib.moe_ep_rows_capacity
@@ -399,6 +402,22 @@ def silu_quant(gate_up: torch.Tensor, recv_src: torch.Tensor, rows_in_use: torch
     act_scale = torch.zeros(shape, dtype=torch.float32, device=gate_up.device)
     silu_quant_into(gate_up, recv_src, rows_in_use, act, act_scale, col_major, stream)
     return act, act_scale
+
+
+def silu_mul(gate: torch.Tensor, up: torch.Tensor, *, exact_only: bool = False,
+             with_fast_value: bool = False, stream: Optional[torch.cuda.Stream] = None):
+    """The activations of moe_silu_quant alone (see moe_silu_mul in the C header):
+    float32 tensor shaped like gate, and with with_fast_value the fp64 values of
+    the kernel's first tier."""
+    g, u = gate.contiguous(), up.contiguous()
+    act = torch.empty(g.shape, dtype=torch.float32, device=g.device)
+    fast = torch.empty(g.shape, dtype=torch.float64, device=g.device) if with_fast_value else None
+    P = ctypes.c_void_p
+    st = lib.moe_silu_mul(g.numel(), P(g.data_ptr()), P(u.data_ptr()), P(act.data_ptr()),
+                          P(fast.data_ptr() if fast is not None else 0), 1 if exact_only else 0,
+                          P(_stream_ptr(stream)))
+    _ok(st, "moe_silu_mul")
+    return (act, fast) if with_fast_value else act
 
 
 def router_topk_into(logits: torch.Tensor, k: int, topk_idx: torch.Tensor, topk_w: torch.Tensor, *,

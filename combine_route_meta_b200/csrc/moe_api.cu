@@ -845,6 +845,30 @@ int moe_silu_quant(int64_t rows_cap, int32_t I, const void *gate_up, const int32
     return launched(launch(silu_quant_rows, grid, kSiluThreads, 0, static_cast<cudaStream_t>(stream), a));
 }
 
+int moe_silu_mul(int64_t n, const void *gate, const void *up, float *act, double *fast_value,
+                 int32_t exact_only, void *stream)
+{
+    if (n < 0)
+        return MOE_ERR_INVALID_ARG;
+    if (n == 0)
+        return MOE_OK;
+    if (gate == nullptr || up == nullptr || act == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    DeviceInfo *dev = nullptr;
+    int st;
+    if ((st = device_info(&dev)) != MOE_OK)
+        return st;
+    SiluMulArgs a;
+    a.gate = static_cast<const uint16_t *>(gate);
+    a.up = static_cast<const uint16_t *>(up);
+    a.n = n;
+    a.act = act;
+    a.fast_value = fast_value;
+    a.exact_only = exact_only ? 1 : 0;
+    const unsigned grid = grid_for((n + kSiluThreads - 1) / kSiluThreads, dev->sms, 8);
+    return launched(launch(silu_mul_values, grid, kSiluThreads, 0, static_cast<cudaStream_t>(stream), a));
+}
+
 int moe_router_topk(int32_t T, int32_t E, int32_t k, const float *logits, int32_t score_fn,
                     int32_t n_group, int32_t topk_group, int32_t renormalize, int32_t *topk_idx,
                     float *topk_w, void *stream)

@@ -276,15 +276,32 @@ MOE_API int moe_combine_rank_partial(const moe_handle *handle, const int32_t *ra
  *   act_scale    fp32 device: [rows_cap, I/128] row-major, or with
  *                scale_col_major != 0, [I/128, rows_cap] (one column of scales
  *                per row, the layout grouped GEMMs read).
- * SiLU(g) = g / (1 + e^-g) in binary32, with e^x by Cody-Waite reduction and a
- * degree-7 Taylor polynomial (fused multiply-adds), -0 below g = -88; the
- * activation is the binary32 product with up.  Per 128 columns: scale =
- * amax/448, codes = e4m3(a/scale) as in moe_dispatch.  I must be a multiple of
- * 128 (else MOE_ERR_UNSUPPORTED).  Rows not selected are left untouched.
+ * The activation a of a (gate g, up u) pair is the binary32 number nearest to
+ * the real value g u / (1 + e^-g) (ties to even; a zero carries the sign of
+ * g u); results beyond the binary32 range are out of contract.  Per 128
+ * columns: scale = amax/448, codes = e4m3(a/scale) as in moe_dispatch.  I must
+ * be a multiple of 128 (else MOE_ERR_UNSUPPORTED).  Rows not selected are left
+ * untouched.
  */
 MOE_API int moe_silu_quant(int64_t rows_cap, int32_t I, const void *gate_up,
                            const int32_t *recv_src, const int32_t *rows_in_use, void *act,
                            float *act_scale, int32_t scale_col_major, void *stream);
+
+/*
+ * The activations of moe_silu_quant alone, for n (gate, up) pairs: act[i] is
+ * the binary32 number nearest to g u / (1 + e^-g) for g = gate[i], u = up[i]
+ * (bf16 device arrays; "Lower latency and higher throughput with multi-node
+ * DeepSeek deployment", section "Quantização": SiLU of the gate times up, the
+ * input of the block quantiser).  The kernel evaluates in fp64 and certifies
+ * the rounding, falling back to double-double arithmetic near a binary32
+ * rounding boundary; exact_only != 0 takes the double-double tier for every
+ * value.  fast_value (fp64 device, may be NULL) receives the fp64 value of the
+ * first tier for each pair (meaningful for finite, nonzero, normal inputs
+ * with gate >= -200), for checking its error bound.  act is fp32 device.
+ * n = 0 launches nothing.  Returns a status.
+ */
+MOE_API int moe_silu_mul(int64_t n, const void *gate, const void *up, float *act,
+                         double *fast_value, int32_t exact_only, void *stream);
 
 /*
  * Router top-k ("Lower latency and higher throughput with multi-node DeepSeek

@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import oracle
-from tests._lib import bf16_from_dev, bf16_to_dev, to_dev
+from tests._lib import bf16_from_dev, bf16_to_dev, silu_pairs_near_rounding_boundaries, to_dev
 from workloads import (WORKLOADS, bf16_bits_to_f32, f32_to_bf16_bits, make_inputs,
                        make_router_logits, normal_bf16_rows, random_problem)
 
@@ -105,7 +105,7 @@ def test_silu_quant_bit_exact(rows, I, in_use, col_major):
 
 
 def test_silu_quant_every_bf16_gate_value():
-    # gate runs through every finite bf16 value (up = 1), so the binary32 SiLU is
+    # gate runs through every finite bf16 value (up = 1), so the activation is
     # checked against the oracle's on its whole input domain
     bits = np.arange(0, 0x10000, dtype=np.uint32)
     bits = bits[((bits >> 7) & 0xFF) != 0xFF].astype(np.uint16)
@@ -118,6 +118,69 @@ def test_silu_quant_every_bf16_gate_value():
     act, sc = moe.silu_quant(bf16_to_dev(gu), to_dev(src), to_dev(np.array([rows], np.int32)))
     np.testing.assert_array_equal(act.view(torch.uint8).cpu().numpy(), act_ref)
     np.testing.assert_array_equal(sc.cpu().numpy().view(np.uint32), sc_ref.view(np.uint32))
+
+
+def _finite_bf16_bits():
+    bits = np.arange(0, 0x10000, dtype=np.uint32)
+    return bits[((bits >> 7) & 0xFF) != 0xFF].astype(np.uint16)
+
+
+def _silu_mul_dev(gb, ub, **kw):
+    return moe.silu_mul(bf16_to_dev(gb), bf16_to_dev(ub), **kw)
+
+
+@pytest.mark.parametrize("exact_only", [False, True])
+def test_silu_activation_every_bf16_gate_value(exact_only):
+    # both tiers of the kernel (certified fp64, and double-double alone) give the
+    # correctly rounded activation on every finite bf16 gate, for up values from
+    # tiny to large
+    bits = _finite_bf16_bits()
+    for ub in (0x3F80, 0xC0A3, 0x0001, 0x0B17, 0x5F3A, 0xF1C4, 0x8000):
+        u = np.full(bits.shape, ub, np.uint16)
+        got = _silu_mul_dev(bits, u, exact_only=exact_only).cpu().numpy()
+        want = oracle.silu_mul_bits(bits, u)
+        bad = np.nonzero(got.view(np.uint32) != want.view(np.uint32))[0]
+        assert bad.size == 0, (hex(ub), [(float(bf16_bits_to_f32(bits[i])), got[i], want[i]) for i in bad[:5]])
+
+
+def test_silu_activation_next_to_rounding_boundaries():
+    # pairs within 2^-36 of a binary32 halfway point: many fall inside the fast
+    # tier's margin, so the double-double tier decides them
+    gb, ub = silu_pairs_near_rounding_boundaries()
+    for shift in (0, 40, -60, -120):
+        us = (ub.astype(np.int32) + (shift << 7)).astype(np.uint16)
+        got, fast = _silu_mul_dev(gb, us, with_fast_value=True)
+        got, fast = got.cpu().numpy(), fast.cpu().numpy()
+        want = oracle.silu_mul_bits(gb, us)
+        np.testing.assert_array_equal(got.view(np.uint32), want.view(np.uint32))
+        low = (fast.view(np.uint64) & np.uint64((1 << 29) - 1)).astype(np.int64)
+        uncertified = np.abs(low - (1 << 28)) <= 32
+        if shift == 0:
+            assert uncertified.sum() > 50          # the exact tier is exercised
+
+
+def test_silu_fast_tier_error_bound():
+    # the fast tier's fp64 value is within 1.25 * 2^-50 (relative) of the real
+    # g u / (1 + e^-g): checked against 50-digit decimal arithmetic on every bf16
+    # gate in [-200, 200] with u = 1, and on pairs next to rounding boundaries
+    from decimal import Context, Decimal
+    ctx = Context(prec=50, Emax=10**6, Emin=-10**6)
+    bits = _finite_bf16_bits()
+    g = bf16_bits_to_f32(bits).astype(np.float64)
+    sel = (g >= -200) & (g <= 200) & (np.abs(g) >= 2.0 ** -126)
+    gb, ub = silu_pairs_near_rounding_boundaries()
+    gb = np.concatenate([bits[sel], gb])
+    ub = np.concatenate([np.full(int(sel.sum()), 0x3F80, np.uint16), ub])
+    _, fast = _silu_mul_dev(gb, ub, with_fast_value=True)
+    fast = fast.cpu().numpy()
+    gv, uv = bf16_bits_to_f32(gb), bf16_bits_to_f32(ub)
+    worst = 0.0
+    for i in range(len(gb)):
+        G, U = Decimal(float(gv[i])), Decimal(float(uv[i]))
+        exact = ctx.divide(ctx.multiply(G, U), ctx.add(1, ctx.exp(-G)))
+        rel = abs((Decimal(float(fast[i])) - exact) / exact)
+        worst = max(worst, float(rel))
+    assert worst <= 1.25 * 2.0 ** -50, worst
 
 
 def test_silu_quant_on_a_dispatch_layout():
