@@ -694,7 +694,12 @@ def run_op(args, peak, peak_kind):
                           y=torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev))
                 rr["out"] = moe.moe_dispatch_out(None, None, b["counts"][r].data_ptr(), rr["off"].data_ptr(),
                                                  rr["roff"].data_ptr(), rr["src"].data_ptr(), S)
+                # completion state: "rows" and "outputs" flags, epochs, CTA count
+                rr["fl_rows"], rr["fl_out"] = torch.zeros(W, **i32), torch.zeros(W, **i32)
+                rr["epochs"], rr["done"] = torch.zeros(2, **i32), torch.zeros(1, **i32)
                 b["r"].append(rr)
+            b["fl_rows"] = [rr["fl_rows"] for rr in b["r"]]
+            b["fl_out"] = [rr["fl_out"] for rr in b["r"]]
             return b
         def ep_step(b):
             P = ctypes.c_void_p
@@ -708,8 +713,14 @@ def run_op(args, peak, peak_kind):
                 moe.ep_layout_into(cfg, r, rr["idx"], rr["slot"], rr["off"], b["counts"], cap, rr["dst"],
                                    rr["rc"], rr["ro"], err, stream)
                 moe.ep_dispatch_payload_into(cfg, rr["x"], rr["idx"], rr["dst"], b["recv_x"],
-                                             b["recv_sc"] if w.fp8 else None, cap, err, stream)
+                                             b["recv_sc"] if w.fp8 else None, cap, err, stream,
+                                             signal=(r, b["fl_rows"], rr["epochs"][0:1], rr["done"]))
             for rr in b["r"]:
+                moe.ep_wait_into(rr["fl_rows"], rr["epochs"][0:1], 1_000_000_000, err, stream)
+            for r, rr in enumerate(b["r"]):
+                moe.ep_signal_into(r, b["fl_out"], rr["epochs"][1:2], stream)
+            for rr in b["r"]:
+                moe.ep_wait_into(rr["fl_out"], rr["epochs"][1:2], 1_000_000_000, err, stream)
                 moe.ep_combine_into(cfg, rr["idx"], rr["dst"], rr["w"], b["eo"], cap, rr["y"], err, stream)
         fn = lambda b: (lambda: ep_step(b))
     else:
@@ -755,7 +766,7 @@ def run_op(args, peak, peak_kind):
         extra = {}
     elif args.op == "ep":
         nbytes = sum(algorithmic_bytes(w.T * w.R, w.H, w.E, w.R, w.k, w.fp8))
-        extra = {"ranks": w.R, "tokens_per_rank": w.T, "kernels_per_launch": 4 * w.R,
+        extra = {"ranks": w.R, "tokens_per_rank": w.T, "kernels_per_launch": 7 * w.R,
                  "note": "virtual ranks on one GPU: local buffers, HBM-bound, no NVLink"}
     else:
         nbytes = w.T * w.E * 4 + S * 8

@@ -119,8 +119,12 @@ def _declare(lib):
     lib.moe_ep_layout.argtypes = [cfgp, i32, i32, P, P, P, P, i64, P, P, P, P, P]
     lib.moe_ep_layout.restype = ctypes.c_int
     lib.moe_ep_dispatch_payload.argtypes = [cfgp, i32, P, P, P, ctypes.POINTER(P), ctypes.POINTER(P),
-                                            i64, P, P]
+                                            i64, i32, ctypes.POINTER(P), P, P, P, P]
     lib.moe_ep_dispatch_payload.restype = ctypes.c_int
+    lib.moe_ep_signal.argtypes = [i32, i32, ctypes.POINTER(P), P, P]
+    lib.moe_ep_signal.restype = ctypes.c_int
+    lib.moe_ep_wait.argtypes = [i32, P, P, ctypes.c_uint64, P, P]
+    lib.moe_ep_wait.restype = ctypes.c_int
     lib.moe_ep_combine.argtypes = [cfgp, i32, P, P, P, ctypes.POINTER(P), i64, P, P, P]
     lib.moe_ep_combine.restype = ctypes.c_int
     lib.moe_check.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
@@ -152,6 +156,8 @@ moe_ep_rows_capacity = lib.moe_ep_rows_capacity
 moe_ep_layout = lib.moe_ep_layout
 moe_ep_dispatch_payload = lib.moe_ep_dispatch_payload
 moe_ep_combine = lib.moe_ep_combine
+moe_ep_signal = lib.moe_ep_signal
+moe_ep_wait = lib.moe_ep_wait
 
 
 class MoeError(RuntimeError):
@@ -514,15 +520,40 @@ def ep_layout_into(cfg: moe_config, rank: int, topk_idx: torch.Tensor, local_slo
 def ep_dispatch_payload_into(cfg: moe_config, x: torch.Tensor, topk_idx: torch.Tensor,
                              dst_row: torch.Tensor, peer_recv_x, peer_recv_scale, rows_cap: int,
                              err: Optional[torch.Tensor] = None,
-                             stream: Optional[torch.cuda.Stream] = None) -> None:
-    """moe_ep_dispatch_payload; the peer tables are W tensors or device addresses."""
+                             stream: Optional[torch.cuda.Stream] = None, signal=None) -> None:
+    """moe_ep_dispatch_payload; the peer tables are W tensors or device addresses.
+    signal = (rank, peer_flags, epoch, done_count) makes the kernel signal the
+    "rows in place" event (see the C header); None signals nothing."""
     P = ctypes.c_void_p
     err = error_word(x.device) if err is None else err
+    rank, flags, epoch, done = (0, None, None, None) if signal is None else signal
     st = lib.moe_ep_dispatch_payload(ctypes.byref(cfg), x.shape[0], P(x.data_ptr()),
                                      P(topk_idx.data_ptr()), P(dst_row.data_ptr()),
                                      _ptr_table(peer_recv_x), _ptr_table(peer_recv_scale), rows_cap,
+                                     rank, _ptr_table(flags),
+                                     P(0 if epoch is None else epoch.data_ptr()),
+                                     P(0 if done is None else done.data_ptr()),
                                      P(err.data_ptr()), P(_stream_ptr(stream)))
     _ok(st, "moe_ep_dispatch_payload")
+
+
+def ep_signal_into(rank: int, peer_flags, epoch: torch.Tensor,
+                   stream: Optional[torch.cuda.Stream] = None) -> None:
+    """moe_ep_signal: publish this rank's next epoch of an event in every peer's flags."""
+    P = ctypes.c_void_p
+    st = lib.moe_ep_signal(len(peer_flags), rank, _ptr_table(peer_flags), P(epoch.data_ptr()),
+                           P(_stream_ptr(stream)))
+    _ok(st, "moe_ep_signal")
+
+
+def ep_wait_into(flags: torch.Tensor, epoch: torch.Tensor, limit_ns: int = 1_000_000_000,
+                 err: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None) -> None:
+    """moe_ep_wait: the stream waits (bounded) until every sender's flag reaches *epoch."""
+    P = ctypes.c_void_p
+    err = error_word(flags.device) if err is None else err
+    st = lib.moe_ep_wait(flags.numel(), P(flags.data_ptr()), P(epoch.data_ptr()), int(limit_ns),
+                         P(err.data_ptr()), P(_stream_ptr(stream)))
+    _ok(st, "moe_ep_wait")
 
 
 def ep_combine_into(cfg: moe_config, topk_idx: torch.Tensor, dst_row: torch.Tensor,

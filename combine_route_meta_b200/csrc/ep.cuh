@@ -26,8 +26,21 @@
 // Peer buffers are reached through a table of W base pointers (peer mappings
 // of the other GPUs' buffers, this rank's own at its index).  Stores and loads
 // are plain 16-byte accesses; nothing here uses TMA or multicast, so the same
-// kernels are correct on peer memory.  Ordering between ranks is the caller's:
-// a stream synchronisation and a barrier between a payload and the peers' reads.
+// kernels are correct on peer memory.
+//
+// Completion (section "Despacho e Combinação": a receiver reads its buffers
+// once the senders have signalled that their writes are complete).  Every rank
+// holds, in its own memory, one int32 flag per sender for each of two events:
+// "the sender's rows are in my receive buffer" and "the sender's expert
+// outputs are ready to be read".  A rank counts its own signals of each event
+// in a device epoch.  To signal, it increments the epoch and stores it, with
+// release semantics at system scope, into its slot of every peer's flags; the
+// payload kernel does this from its last CTA, after every CTA has fenced its
+// stores at system scope and counted itself done.  To wait, a rank polls its
+// own flags with acquire loads until each reaches its own epoch of the event
+// (every rank signals each event once per layer, so the epochs agree), for a
+// bounded time; on expiry it sets MOE_DEV_TIMEOUT and returns.  The host never
+// blocks, so a layer's exchange can be captured in a CUDA graph.
 #pragma once
 
 #include "combine.cuh"
@@ -110,6 +123,89 @@ __global__ void __launch_bounds__(kEpThreads) ep_rows(EpRowsArgs a)
     }
 }
 
+// ---- completion flags ---------------------------------------------------------
+
+struct EpFlagPeers {
+    int32_t *p[kEpMaxRanks]; // [W] each rank's flags of one event, W int32 each
+};
+
+// A sender's side of one event: its slot `rank` in every peer's flags, its
+// epoch of the event, and (payload kernel only) the count of CTAs done.
+struct EpSignal {
+    EpFlagPeers flags;
+    int32_t *epoch;
+    int32_t *done;
+    int32_t rank, W;
+    int32_t enabled;
+};
+
+__device__ __forceinline__ void st_release_sys(int32_t *p, int32_t v)
+{
+    asm volatile("st.release.sys.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ int32_t ld_acquire_sys(const int32_t *p)
+{
+    int32_t v;
+    asm volatile("ld.acquire.sys.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// One thread: makes this grid's earlier writes visible at system scope, then
+// publishes the next epoch in every peer's slot of this sender.
+__device__ __forceinline__ void ep_publish(const EpSignal &s)
+{
+    __threadfence_system();
+    const int32_t e = *s.epoch + 1;
+    *s.epoch = e;
+    for (int32_t d = 0; d < s.W; ++d)
+        st_release_sys(s.flags.p[d] + s.rank, e);
+}
+
+// End of a grid whose writes the signal covers: every CTA fences its threads'
+// writes at system scope and counts itself done; the last CTA publishes.  The
+// count is reset for the next launch, which stream order puts after this one.
+__device__ __forceinline__ void ep_signal_grid(const EpSignal &s)
+{
+    __threadfence_system();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const int32_t prev = atomicAdd(s.done, 1);
+        if (prev == (int32_t)gridDim.x - 1) {
+            *s.done = 0;
+            ep_publish(s);
+        }
+    }
+}
+
+// moe_ep_signal: publishes after the previous kernel in the stream completed.
+__global__ void __launch_bounds__(kWarp) ep_signal(EpSignal s)
+{
+    stream_order_begin();
+    if (threadIdx.x == 0)
+        ep_publish(s);
+}
+
+// moe_ep_wait: until flags[s] reaches *epoch for every sender s (wrap-safe
+// comparison), each polled by one thread, for at most limit_ns in all.
+__global__ void __launch_bounds__(kEpThreads) ep_wait(const int32_t *flags, const int32_t *epoch, int32_t W,
+                                                      uint64_t limit_ns, int32_t *err)
+{
+    stream_order_begin();
+    const int32_t target = *epoch;
+    const uint64_t t0 = global_ns();
+    for (int32_t s = threadIdx.x; s < W; s += blockDim.x) {
+        // the difference is taken in unsigned arithmetic, which wraps
+        while ((int32_t)((uint32_t)ld_acquire_sys(flags + s) - (uint32_t)target) < 0) {
+            if (global_ns() - t0 > limit_ns) {
+                raise_error(err, MOE_DEV_TIMEOUT);
+                break;
+            }
+            __nanosleep(100);
+        }
+    }
+}
+
 struct EpPayloadArgs {
     const uint16_t *x;
     const int32_t *topk_idx, *dst_row;
@@ -117,6 +213,7 @@ struct EpPayloadArgs {
     int64_t rows_cap;
     EpPeers recv_x;     // [W] receive buffers [rows_cap, H]
     EpPeers recv_scale; // [W] fp8 scales [rows_cap, H/128]
+    EpSignal sig;       // "rows in place", when enabled
     int32_t *err;
 };
 
@@ -193,6 +290,8 @@ __global__ void __launch_bounds__(kScatterThreads) ep_payload(EpPayloadArgs a)
             }
         }
     }
+    if (a.sig.enabled)
+        ep_signal_grid(a.sig);
 }
 
 struct EpCombineArgs {

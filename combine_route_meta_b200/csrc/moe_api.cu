@@ -969,23 +969,40 @@ int moe_ep_layout(const moe_config *cfg, int32_t rank, int32_t T, const int32_t 
 
 int moe_ep_dispatch_payload(const moe_config *cfg, int32_t T, const void *x, const int32_t *topk_idx,
                             const int32_t *dst_row, void *const *peer_recv_x,
-                            float *const *peer_recv_scale, int64_t rows_cap, int32_t *dev_err,
-                            void *stream)
+                            float *const *peer_recv_scale, int64_t rows_cap, int32_t rank,
+                            int32_t *const *peer_flags, int32_t *epoch, int32_t *done_count,
+                            int32_t *dev_err, void *stream)
 {
     int st = check_ep(cfg, T, rows_cap);
     if (st != MOE_OK)
         return st;
     const bool fp8 = cfg->flags & MOE_FP8;
+    const bool signal = peer_flags != nullptr;
     if (dev_err == nullptr)
         return MOE_ERR_INVALID_ARG;
-    if (T == 0)
+    if (signal && (rank < 0 || rank >= cfg->R || epoch == nullptr || done_count == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0 && !signal)
         return MOE_OK;
-    if (x == nullptr || !aligned16(x) || topk_idx == nullptr || dst_row == nullptr)
+    if (T > 0 && (x == nullptr || !aligned16(x) || topk_idx == nullptr || dst_row == nullptr))
         return MOE_ERR_INVALID_ARG;
     EpPayloadArgs a;
-    if ((st = fill_peers(&a.recv_x, (const void *const *)peer_recv_x, cfg->R, true)) != MOE_OK ||
-        (st = fill_peers(&a.recv_scale, (const void *const *)peer_recv_scale, cfg->R, fp8)) != MOE_OK)
+    if ((st = fill_peers(&a.recv_x, (const void *const *)peer_recv_x, cfg->R, T > 0)) != MOE_OK ||
+        (st = fill_peers(&a.recv_scale, (const void *const *)peer_recv_scale, cfg->R, T > 0 && fp8)) != MOE_OK)
         return st;
+    a.sig.enabled = signal ? 1 : 0;
+    a.sig.rank = rank;
+    a.sig.W = cfg->R;
+    a.sig.epoch = epoch;
+    a.sig.done = done_count;
+    for (int32_t r = 0; r < kEpMaxRanks; ++r)
+        a.sig.flags.p[r] = nullptr;
+    if (signal)
+        for (int32_t r = 0; r < cfg->R; ++r) {
+            if (peer_flags[r] == nullptr)
+                return MOE_ERR_INVALID_ARG;
+            a.sig.flags.p[r] = peer_flags[r];
+        }
     DeviceInfo *dev = nullptr;
     if ((st = device_info(&dev)) != MOE_OK)
         return st;
@@ -1003,9 +1020,41 @@ int moe_ep_dispatch_payload(const moe_config *cfg, int32_t T, const void *x, con
                                         chunk_cols<kScatterLaneCols>());
     const int64_t ctas = (units + kScatterThreads / kWarp - 1) / (kScatterThreads / kWarp);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const cudaError_t e = fp8 ? launch(ep_payload<true>, grid_for(ctas, dev->sms, 8), kScatterThreads, 0, s, a)
-                              : launch(ep_payload<false>, grid_for(ctas, dev->sms, 8), kScatterThreads, 0, s, a);
+    // with T == 0 one CTA still runs, to signal
+    const unsigned grid = grid_for(ctas, dev->sms, 8);
+    const cudaError_t e = fp8 ? launch(ep_payload<true>, grid, kScatterThreads, 0, s, a)
+                              : launch(ep_payload<false>, grid, kScatterThreads, 0, s, a);
     return launched(e);
+}
+
+int moe_ep_signal(int32_t W, int32_t rank, int32_t *const *peer_flags, int32_t *epoch, void *stream)
+{
+    if (W <= 0 || W > kEpMaxRanks || rank < 0 || rank >= W || peer_flags == nullptr || epoch == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    EpSignal sig;
+    for (int32_t r = 0; r < kEpMaxRanks; ++r)
+        sig.flags.p[r] = nullptr;
+    for (int32_t r = 0; r < W; ++r) {
+        if (peer_flags[r] == nullptr)
+            return MOE_ERR_INVALID_ARG;
+        sig.flags.p[r] = peer_flags[r];
+    }
+    sig.epoch = epoch;
+    sig.done = nullptr;
+    sig.rank = rank;
+    sig.W = W;
+    sig.enabled = 1;
+    return launched(launch(ep_signal, 1, kWarp, 0, static_cast<cudaStream_t>(stream), sig));
+}
+
+int moe_ep_wait(int32_t W, const int32_t *flags, const int32_t *epoch, uint64_t limit_ns,
+                int32_t *dev_err, void *stream)
+{
+    if (W <= 0 || W > kEpMaxRanks || flags == nullptr || epoch == nullptr || dev_err == nullptr ||
+        limit_ns == 0 || limit_ns > MOE_EP_MAX_WAIT_NS)
+        return MOE_ERR_INVALID_ARG;
+    return launched(launch(ep_wait, 1, kEpThreads, 0, static_cast<cudaStream_t>(stream), flags, epoch, W,
+                           limit_ns, dev_err));
 }
 
 int moe_ep_combine(const moe_config *cfg, int32_t T, const int32_t *topk_idx, const int32_t *dst_row,

@@ -70,7 +70,7 @@ extern "C" {
 /* Bits of the device error word. */
 #define MOE_DEV_BAD_INDEX 1 /* dispatch: an expert id outside [0, E)                  */
 #define MOE_DEV_CAPACITY 2  /* dispatch: a receive row at or past rows_cap            */
-#define MOE_DEV_TIMEOUT 4   /* a bounded device wait (1 s) gave up                     */
+#define MOE_DEV_TIMEOUT 4   /* a bounded device wait gave up                           */
 #define MOE_DEV_BAD_SLOT 8  /* payload / combine: a slot outside [-1, rows_cap)        */
 
 /* Router score functions (moe_router_topk). */
@@ -81,6 +81,7 @@ extern "C" {
 #define MOE_MAX_EXPERTS 2048 /* E */
 #define MOE_MAX_TOPK 64      /* k */
 #define MOE_NO_ALLOC_SCRATCH_BYTES (1u << 20) /* fixed scratch of moe_dispatch_no_alloc */
+#define MOE_EP_MAX_WAIT_NS 10000000000ull   /* longest moe_ep_wait limit: 10 s      */
 
 /*
  * Problem description.
@@ -292,10 +293,10 @@ MOE_API int moe_silu_quant(int64_t rows_cap, int32_t I, const void *gate_up,
  * the binary32 number nearest to g u / (1 + e^-g) for g = gate[i], u = up[i]
  * (bf16 device arrays; "Lower latency and higher throughput with multi-node
  * DeepSeek deployment", section "Quantização": SiLU of the gate times up, the
- * input of the block quantiser).  The kernel evaluates in fp64 and certifies
- * the rounding, falling back to double-double arithmetic near a binary32
- * rounding boundary; exact_only != 0 takes the double-double tier for every
- * value.  fast_value (fp64 device, may be NULL) receives the fp64 value of the
+ * input of the block quantiser).  The kernel evaluates g u sigmoid(g) in fp64
+ * (sigmoid from a per-CTA table for common gates) and certifies the rounding,
+ * falling back to double-double arithmetic near a binary32 rounding boundary;
+ * exact_only != 0 takes the double-double tier for every value.  fast_value (fp64 device, may be NULL) receives the fp64 value of the
  * first tier for each pair (meaningful for finite, nonzero, normal inputs
  * with gate >= -200), for checking its error bound.  act is fp32 device.
  * n = 0 launches nothing.  Returns a status.
@@ -358,9 +359,15 @@ MOE_API int moe_route_dispatch(const moe_config *cfg, int32_t T, const void *x,
  *      counts, offsets and slots);
  *   2. an all-gather of the E counts into counts_all[W, E] (the caller's
  *      collective, e.g. NCCL);
- *   3. moe_ep_layout, then moe_ep_dispatch_payload with the W receive buffers;
- *   4. after a barrier that orders every rank's payload before the experts
- *      read, and after the experts, moe_ep_combine with the W expert outputs.
+ *   3. moe_ep_layout, then moe_ep_dispatch_payload with the W receive buffers
+ *      and the "rows" flags, then moe_ep_wait on its own "rows" flags: the
+ *      rank's buffer then holds every sender's rows;
+ *   4. after its experts wrote their outputs, moe_ep_signal on the "outputs"
+ *      flags, then moe_ep_wait on its own "outputs" flags, then moe_ep_combine
+ *      with the W expert outputs.
+ * No step blocks the host, so a layer's exchange can be captured in a CUDA
+ * graph (section "Despacho e Combinação": a receiver uses its buffers once the
+ * senders have signalled completion).
  * Buffer tables are host arrays of W device pointers (peer mappings; the
  * rank's own buffer at its index), each 16-byte aligned, every buffer
  * [rows_cap, H] (and [rows_cap, H/128] scales for fp8).  The kernels use plain
@@ -379,7 +386,26 @@ MOE_API int moe_route_dispatch(const moe_config *cfg, int32_t T, const void *x,
  * moe_ep_dispatch_payload: copies (bf16) or quantises (MOE_FP8, as
  * moe_dispatch does) x[t] into row dst_row[t,j] of the buffer of the rank that
  * hosts topk_idx[t,j].  Rows outside [-1, rows_cap) set MOE_DEV_BAD_SLOT and are
- * skipped.
+ * skipped.  With peer_flags non-NULL (a host table of W device pointers, each
+ * rank's "rows" flags: W int32 per rank, zero before the first layer), the
+ * kernel's last CTA, once every CTA's stores are visible at system scope,
+ * increments *epoch (an int32 in this rank's memory, zero before the first
+ * layer) and stores the new value into peer_flags[d][rank] of every rank d,
+ * with release semantics at system scope; *done_count (an int32 in this
+ * rank's memory, zero before the first layer) counts the finished CTAs and is
+ * left at zero.  It signals with T = 0 too.
+ *
+ * moe_ep_signal: once the previous kernel in the stream has completed,
+ * increments *epoch and stores it into peer_flags[d][rank] for every rank d
+ * (release, system scope): the same signal without a payload, for the
+ * "outputs" event after the experts.
+ *
+ * moe_ep_wait: waits until flags[s] >= *epoch for every sender s < W (flags
+ * and epoch in this rank's memory; acquire loads at system scope, wrap-safe
+ * comparison) for at most limit_ns (1 ns .. MOE_EP_MAX_WAIT_NS) in all; on
+ * expiry it sets MOE_DEV_TIMEOUT in *dev_err and returns, so the stream goes
+ * on and the caller learns of it from moe_check.  Kernels after it in the
+ * stream see every waited-for sender's writes.
  *
  * moe_ep_combine: y[t] = bf16(sum_j w[t,j] * row dst_row[t,j] of the expert
  * output of the rank hosting topk_idx[t,j]), the fp32 chain of moe_combine.
@@ -395,7 +421,13 @@ MOE_API int moe_ep_layout(const moe_config *cfg, int32_t rank, int32_t T, const 
 MOE_API int moe_ep_dispatch_payload(const moe_config *cfg, int32_t T, const void *x,
                                     const int32_t *topk_idx, const int32_t *dst_row,
                                     void *const *peer_recv_x, float *const *peer_recv_scale,
-                                    int64_t rows_cap, int32_t *dev_err, void *stream);
+                                    int64_t rows_cap, int32_t rank, int32_t *const *peer_flags,
+                                    int32_t *epoch, int32_t *done_count, int32_t *dev_err,
+                                    void *stream);
+MOE_API int moe_ep_signal(int32_t W, int32_t rank, int32_t *const *peer_flags, int32_t *epoch,
+                          void *stream);
+MOE_API int moe_ep_wait(int32_t W, const int32_t *flags, const int32_t *epoch, uint64_t limit_ns,
+                        int32_t *dev_err, void *stream);
 MOE_API int moe_ep_combine(const moe_config *cfg, int32_t T, const int32_t *topk_idx,
                            const int32_t *dst_row, const float *topk_w,
                            const void *const *peer_expert_out, int64_t rows_cap, void *y,

@@ -130,14 +130,29 @@ def test_expert_parallel_calls_check_their_arguments():
                              None) == moe.ERR_UNSUPPORTED
     table = (P * 4)(16, 32, None, 48)                                 # a missing peer buffer
     assert moe.moe_ep_dispatch_payload(ctypes.byref(cfg), 10, P(16), P(16), P(16), table, None, 100,
-                                       P(16), None) == moe.ERR_INVALID_ARG
+                                       0, None, None, None, P(16), None) == moe.ERR_INVALID_ARG
     table = (P * 4)(16, 32, 40, 48)                                   # a misaligned one
     assert moe.moe_ep_dispatch_payload(ctypes.byref(cfg), 10, P(16), P(16), P(16), table, None, 100,
-                                       P(16), None) == moe.ERR_INVALID_ARG
+                                       0, None, None, None, P(16), None) == moe.ERR_INVALID_ARG
     f8 = moe.make_config(256, 2, 16, 4, fp8=True)                     # fp8 without scale buffers
     table = (P * 4)(16, 32, 64, 48)
     assert moe.moe_ep_dispatch_payload(ctypes.byref(f8), 10, P(16), P(16), P(16), table, None, 100,
-                                       P(16), None) == moe.ERR_INVALID_ARG
+                                       0, None, None, None, P(16), None) == moe.ERR_INVALID_ARG
+    flags = (P * 4)(16, 32, 64, 48)
+    # signalling: rank outside [0, W), missing epoch or done count, a missing peer flag array
+    for rank, ep, done, fl in [(4, P(16), P(16), flags), (0, None, P(16), flags), (0, P(16), None, flags),
+                               (0, P(16), P(16), (P * 4)(16, None, 64, 48))]:
+        assert moe.moe_ep_dispatch_payload(ctypes.byref(cfg), 0, None, None, None, None, None, 100,
+                                           rank, fl, ep, done, P(16), None) == moe.ERR_INVALID_ARG
+    assert moe.moe_ep_signal(0, 0, flags, P(16), None) == moe.ERR_INVALID_ARG
+    assert moe.moe_ep_signal(4, 4, flags, P(16), None) == moe.ERR_INVALID_ARG
+    assert moe.moe_ep_signal(4, 0, (P * 4)(16, 32, None, 48), P(16), None) == moe.ERR_INVALID_ARG
+    assert moe.moe_ep_signal(4, 0, flags, None, None) == moe.ERR_INVALID_ARG
+    assert moe.moe_ep_wait(4, P(16), P(16), 0, P(16), None) == moe.ERR_INVALID_ARG
+    assert moe.moe_ep_wait(4, P(16), P(16), 10_000_000_001, P(16), None) == moe.ERR_INVALID_ARG
+    assert moe.moe_ep_wait(65, P(16), P(16), 1000, P(16), None) == moe.ERR_INVALID_ARG
+    assert moe.moe_ep_wait(4, None, P(16), 1000, P(16), None) == moe.ERR_INVALID_ARG
+    assert moe.moe_ep_wait(4, P(16), P(16), 1000, None, None) == moe.ERR_INVALID_ARG
     assert moe.moe_ep_combine(ctypes.byref(cfg), 10, P(16), P(16), P(16), None, 100, P(16), P(16),
                               None) == moe.ERR_INVALID_ARG
     assert moe.moe_ep_combine(ctypes.byref(cfg), 10, P(16), P(16), P(16), table, -1, P(16), P(16),

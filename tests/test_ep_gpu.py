@@ -6,8 +6,10 @@ addressing is exactly that of W GPUs writing into each other's buffers.  Rank
 d's buffer must equal rows [rank_offset[d], rank_offset[d+1]) of the oracle's
 single-GPU dispatch of all ranks' batches concatenated in rank order (R = W),
 and each rank's combine must equal, bit for bit, the single-GPU combine of the
-concatenated batch for its tokens.  A one-rank NCCL group runs the host
-orchestration (count exchange, buffer sharing, barriers) end to end.
+concatenated batch for its tokens.  The ranks' completion flags are exercised
+in the one stream (all payloads, which signal, before all waits).  A one-rank
+NCCL group runs the host orchestration (count exchange, buffer sharing,
+device-side completion, graph capture) end to end.
 """
 import os
 import socket
@@ -46,7 +48,14 @@ def _local_layout(H, k, E, idx_dev):
     return buf.expert_count, buf.expert_offset, buf.slot
 
 
-def _run_ep(W, E, k, H, Ts, fp8, pad, seed, bad_ids=False, rows_cap=None):
+def _signals(W):
+    """Every virtual rank's completion state: its "rows" flags (one per sender),
+    its epoch of the event and its payload's CTA count, all zero."""
+    z = lambda n: torch.zeros(n, dtype=torch.int32, device="cuda")
+    return dict(flags=[z(W) for _ in range(W)], epoch=[z(1) for _ in range(W)], done=[z(1) for _ in range(W)])
+
+
+def _run_ep(W, E, k, H, Ts, fp8, pad, seed, bad_ids=False, rows_cap=None, layers=1):
     batches = [random_problem(seed + r, T, H, E, k) for r, T in enumerate(Ts)]
     if bad_ids:
         batches[0][1][0, 0] = E          # out of range
@@ -61,17 +70,28 @@ def _run_ep(W, E, k, H, Ts, fp8, pad, seed, bad_ids=False, rows_cap=None):
     recv_x = [_poisoned(cap, H, torch.uint8 if fp8 else torch.int16) for _ in range(W)]
     recv_sc = [_poisoned(cap, H // 128, torch.float32) for _ in range(W)] if fp8 else None
     El = E // W
-    dst, rcount, roff = [], [], []
-    for r in range(W):
-        d = torch.empty_like(locals_[r][2])
-        rc = torch.empty(El, dtype=torch.int32, device="cuda")
-        ro = torch.empty(El + 1, dtype=torch.int32, device="cuda")
-        moe.ep_layout_into(cfg, r, idxs[r], locals_[r][2], locals_[r][1], counts_all, cap, d, rc, ro)
-        moe.ep_dispatch_payload_into(cfg, xs[r], idxs[r], d, recv_x, recv_sc, cap)
-        dst.append(d)
-        rcount.append(rc)
-        roff.append(ro)
-    torch.cuda.synchronize()
+    sig = _signals(W)
+    for layer in range(layers):
+        dst, rcount, roff = [], [], []
+        # every sender's payload signals "rows in place" in every rank's flags;
+        # the waits come after all payloads in the one stream, so none waits
+        # on a kernel that has not run
+        for r in range(W):
+            d = torch.empty_like(locals_[r][2])
+            rc = torch.empty(El, dtype=torch.int32, device="cuda")
+            ro = torch.empty(El + 1, dtype=torch.int32, device="cuda")
+            moe.ep_layout_into(cfg, r, idxs[r], locals_[r][2], locals_[r][1], counts_all, cap, d, rc, ro)
+            moe.ep_dispatch_payload_into(cfg, xs[r], idxs[r], d, recv_x, recv_sc, cap,
+                                         signal=(r, sig["flags"], sig["epoch"][r], sig["done"][r]))
+            dst.append(d)
+            rcount.append(rc)
+            roff.append(ro)
+        for r in range(W):
+            moe.ep_wait_into(sig["flags"][r], sig["epoch"][r], 1_000_000_000)
+        torch.cuda.synchronize()
+        for r in range(W):
+            assert sig["flags"][r].cpu().tolist() == [layer + 1] * W
+            assert int(sig["epoch"][r].item()) == layer + 1 and int(sig["done"][r].item()) == 0
     return dict(batches=batches, cfg=cfg, cap=cap, xs=xs, idxs=idxs, ws=ws, dst=dst, rcount=rcount,
                 roff=roff, recv_x=recv_x, recv_sc=recv_sc)
 
@@ -85,7 +105,7 @@ def _run_ep(W, E, k, H, Ts, fp8, pad, seed, bad_ids=False, rows_cap=None):
 ])
 def test_ep_matches_the_concatenated_single_gpu_dispatch(W, E, k, H, Ts, fp8, pad, bad):
     moe.check()
-    run = _run_ep(W, E, k, H, Ts, fp8, pad, seed=W * 100 + E, bad_ids=bad)
+    run = _run_ep(W, E, k, H, Ts, fp8, pad, seed=W * 100 + E, bad_ids=bad, layers=2)
     assert moe.check() == (moe.DEV_BAD_INDEX if bad else 0)
     X = np.concatenate([b[0] for b in run["batches"]])
     IDX = np.concatenate([b[1] for b in run["batches"]])
@@ -114,7 +134,13 @@ def test_ep_matches_the_concatenated_single_gpu_dispatch(W, E, k, H, Ts, fp8, pa
             gs = run["recv_sc"][d].view(torch.uint8).cpu().numpy().reshape(run["cap"], -1)
             rs = o["recv_scale"].view(np.uint8).reshape(o["recv_scale"].shape[0], -1)[ro[d]:ro[d + 1]]
             np.testing.assert_array_equal(gs[:n], rs)
-    # combine: each rank reads its rows from the hosting ranks' expert outputs
+    # combine: each rank reads its rows from the hosting ranks' expert outputs,
+    # after every rank signalled "outputs ready" and waited for the others
+    out_sig = _signals(W)
+    for r in range(W):
+        moe.ep_signal_into(r, out_sig["flags"], out_sig["epoch"][r])
+    for r in range(W):
+        moe.ep_wait_into(out_sig["flags"][r], out_sig["epoch"][r], 1_000_000_000)
     rows_g = o["recv_x"].shape[0]
     eo_g = normal_bf16_rows(5, 3, 0, rows_g, H)
     eo = []
@@ -160,6 +186,37 @@ def test_ep_capacity_overflow_stays_inside_the_buffers():
     assert moe.check() & moe.DEV_CAPACITY
 
 
+def test_ep_wait_gives_up_on_a_flag_nothing_sets():
+    # a sender that never signals: the wait runs out after its limit, sets the
+    # timeout bit and returns, and the stream and context stay usable
+    moe.check()
+    flags = torch.zeros(4, dtype=torch.int32, device="cuda")
+    flags[:3] = 1                                    # sender 3 never signals
+    epoch = torch.ones(1, dtype=torch.int32, device="cuda")
+    moe.ep_wait_into(flags, epoch, 2_000_000)        # 2 ms
+    assert moe.check() == moe.DEV_TIMEOUT
+    flags[3] = 1
+    moe.ep_wait_into(flags, epoch, 2_000_000)
+    assert moe.check() == 0
+    x, idx, w = random_problem(1, 64, 256, 8, 2)     # ordinary work afterwards
+    d = moe.dispatch(bf16_to_dev(x), to_dev(idx), to_dev(w), 8, 2, False)
+    o = oracle.dispatch(x, idx, E=8, R=2, fp8=False)
+    np.testing.assert_array_equal(d.handle.slot.cpu().numpy(), o["slot"])
+    assert moe.check() == 0
+
+
+def test_ep_signal_wraps_its_epoch_comparison():
+    # epochs compare wrap-safe: a flag one past the int32 maximum still counts
+    flags = torch.tensor([-2**31, 2**31 - 1], dtype=torch.int32, device="cuda")
+    epoch = torch.tensor([2**31 - 1], dtype=torch.int32, device="cuda")
+    moe.check()
+    moe.ep_wait_into(flags, epoch, 2_000_000)
+    assert moe.check() == 0
+    flags[1] = 2**31 - 2
+    moe.ep_wait_into(flags, epoch, 2_000_000)
+    assert moe.check() == moe.DEV_TIMEOUT
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
@@ -189,12 +246,49 @@ got = ep.recv_x.view(torch.uint8).cpu().numpy()[:n]
 assert np.array_equal(got[valid], o["recv_x"][:n][valid])
 eo = normal_bf16_rows(4, 3, 0, ep.rows_cap, 1024)
 ep.expert_out.copy_(bf16_to_dev(eo))
+ep.experts_done()
 y = ep.combine(to_dev(idx), dst, to_dev(w))
 ref = oracle.combine(o["slot"], w, eo[:o["recv_x"].shape[0]])
 yf = bf16_from_dev(y).astype(np.uint32) << 16
 err = np.abs(yf.view(np.float32).astype(np.float64) - ref)
 assert np.all(err <= 1e-2 + 4e-3 * np.abs(ref))
-assert moe.check() == 0
+ep.check()
+# the whole layer (layout, count exchange, payload, waits, signals, combine)
+# captured in a CUDA graph and replayed: the same result, epochs advancing
+xd, idd, wd = bf16_to_dev(x), to_dev(idx), to_dev(w)
+s = torch.cuda.Stream()
+s.wait_stream(torch.cuda.current_stream())
+with torch.cuda.stream(s):
+    for _ in range(2):   # warm-up outside capture
+        dd = ep.dispatch(xd, idd); ep.experts_done(); yy = ep.combine(idd, dd, wd)
+torch.cuda.current_stream().wait_stream(s)
+torch.cuda.synchronize()
+e0 = ep.epochs.cpu().tolist()
+g = torch.cuda.CUDAGraph()
+with torch.cuda.graph(g):
+    dg = ep.dispatch(xd, idd)
+    ep.experts_done()
+    yg = ep.combine(idd, dg, wd)
+for _ in range(3):
+    g.replay()
+torch.cuda.synchronize()
+assert ep.epochs.cpu().tolist() == [e0[0] + 3, e0[1] + 3]     # capture records, replays run
+assert np.array_equal(bf16_from_dev(yg), bf16_from_dev(y))
+ep.check()
+del g
+# a batch above T_max is refused on the host; a bad id is reported by check()
+try:
+    ep.dispatch(bf16_to_dev(np.zeros((201, 1024), np.uint16)), to_dev(np.zeros((201, 4), np.int32)))
+    raise AssertionError("T > T_max accepted")
+except ValueError:
+    pass
+bad = idx.copy(); bad[0, 0] = 99
+ep.dispatch(xd, to_dev(bad)); ep.experts_done(); ep.combine(to_dev(bad), dst, wd)
+try:
+    ep.check()
+    raise AssertionError("bad id not reported")
+except moe.MoeError:
+    pass
 del ep
 dist.destroy_process_group()
 print("ONE RANK OK")

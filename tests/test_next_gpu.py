@@ -160,7 +160,7 @@ def test_silu_activation_next_to_rounding_boundaries():
 
 
 def test_silu_fast_tier_error_bound():
-    # the fast tier's fp64 value is within 1.25 * 2^-50 (relative) of the real
+    # the fast tier's fp64 value is within 1.5 * 2^-50 (relative) of the real
     # g u / (1 + e^-g): checked against 50-digit decimal arithmetic on every bf16
     # gate in [-200, 200] with u = 1, and on pairs next to rounding boundaries
     from decimal import Context, Decimal
@@ -180,7 +180,7 @@ def test_silu_fast_tier_error_bound():
         exact = ctx.divide(ctx.multiply(G, U), ctx.add(1, ctx.exp(-G)))
         rel = abs((Decimal(float(fast[i])) - exact) / exact)
         worst = max(worst, float(rel))
-    assert worst <= 1.25 * 2.0 ** -50, worst
+    assert worst <= 1.5 * 2.0 ** -50, worst
 
 
 def test_silu_quant_on_a_dispatch_layout():
