@@ -33,11 +33,12 @@
 // holds, in its own memory, one int32 flag per sender for each of two events:
 // "the sender's rows are in my receive buffer" and "the sender's expert
 // outputs are ready to be read".  A rank counts its own signals of each event
-// in a device epoch.  To signal, it increments the epoch and stores it, with
-// release semantics at system scope, into its slot of every peer's flags; the
-// payload kernel does this from its last CTA, after every CTA has fenced its
-// stores at system scope and counted itself done.  To wait, a rank polls its
-// own flags with acquire loads until each reaches its own epoch of the event
+// in a device epoch.  To signal, it fences at system scope, increments the
+// epoch and stores it into its slot of every peer's flags (a release pattern);
+// the payload kernel does this from its last CTA, after every CTA has fenced
+// its stores at system scope and counted itself done.  To wait, a rank polls
+// its own flags until each reaches its own epoch of the event, then fences (an
+// acquire pattern)
 // (every rank signals each event once per layer, so the epochs agree), for a
 // bounded time; on expiry it sets MOE_DEV_TIMEOUT and returns.  The host never
 // blocks, so a layer's exchange can be captured in a CUDA graph.
@@ -139,15 +140,18 @@ struct EpSignal {
     int32_t enabled;
 };
 
-__device__ __forceinline__ void st_release_sys(int32_t *p, int32_t v)
+// Relaxed system-scope accesses: with one fence before the stores (a release
+// pattern) and one after the loads (an acquire pattern), a signal costs one
+// system-scope fence however many peers it reaches or polls.
+__device__ __forceinline__ void st_relaxed_sys(int32_t *p, int32_t v)
 {
-    asm volatile("st.release.sys.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+    asm volatile("st.relaxed.sys.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ int32_t ld_acquire_sys(const int32_t *p)
+__device__ __forceinline__ int32_t ld_relaxed_sys(const int32_t *p)
 {
     int32_t v;
-    asm volatile("ld.acquire.sys.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    asm volatile("ld.relaxed.sys.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
 
@@ -159,17 +163,19 @@ __device__ __forceinline__ void ep_publish(const EpSignal &s)
     const int32_t e = *s.epoch + 1;
     *s.epoch = e;
     for (int32_t d = 0; d < s.W; ++d)
-        st_release_sys(s.flags.p[d] + s.rank, e);
+        st_relaxed_sys(s.flags.p[d] + s.rank, e);
 }
 
-// End of a grid whose writes the signal covers: every CTA fences its threads'
-// writes at system scope and counts itself done; the last CTA publishes.  The
-// count is reset for the next launch, which stream order puts after this one.
+// End of a grid whose writes the signal covers: the CTA's barrier orders its
+// threads' writes before thread 0, whose system-scope fence (cumulative over
+// what the barrier ordered before it) precedes its count of the CTA as done;
+// the last CTA to count publishes.  The count is reset for the next launch,
+// which stream order puts after this one.
 __device__ __forceinline__ void ep_signal_grid(const EpSignal &s)
 {
-    __threadfence_system();
     __syncthreads();
     if (threadIdx.x == 0) {
+        __threadfence_system();
         const int32_t prev = atomicAdd(s.done, 1);
         if (prev == (int32_t)gridDim.x - 1) {
             *s.done = 0;
@@ -187,7 +193,8 @@ __global__ void __launch_bounds__(kWarp) ep_signal(EpSignal s)
 }
 
 // moe_ep_wait: until flags[s] reaches *epoch for every sender s (wrap-safe
-// comparison), each polled by one thread, for at most limit_ns in all.
+// comparison), each polled by one thread, for at most limit_ns in all; then a
+// system-scope fence.
 __global__ void __launch_bounds__(kEpThreads) ep_wait(const int32_t *flags, const int32_t *epoch, int32_t W,
                                                       uint64_t limit_ns, int32_t *err)
 {
@@ -196,7 +203,7 @@ __global__ void __launch_bounds__(kEpThreads) ep_wait(const int32_t *flags, cons
     const uint64_t t0 = global_ns();
     for (int32_t s = threadIdx.x; s < W; s += blockDim.x) {
         // the difference is taken in unsigned arithmetic, which wraps
-        while ((int32_t)((uint32_t)ld_acquire_sys(flags + s) - (uint32_t)target) < 0) {
+        while ((int32_t)((uint32_t)ld_relaxed_sys(flags + s) - (uint32_t)target) < 0) {
             if (global_ns() - t0 > limit_ns) {
                 raise_error(err, MOE_DEV_TIMEOUT);
                 break;
@@ -204,6 +211,7 @@ __global__ void __launch_bounds__(kEpThreads) ep_wait(const int32_t *flags, cons
             __nanosleep(100);
         }
     }
+    __threadfence_system(); // the peers' writes before their signals are seen after this kernel
 }
 
 struct EpPayloadArgs {
