@@ -260,7 +260,7 @@ def graph_kernels(g):
 
 def short_kernel_name(mangled):
     for k in ("dispatch_fused", "dispatch_direct", "dispatch_multi", "scatter_bulk_bf16",
-              "scatter_rows", "combine_rows", "meta_single_block", "meta_tile_count",
+              "scatter_bulk_fp8", "scatter_rows", "combine_rows", "meta_single_block", "meta_tile_count",
               "meta_tile_scan", "meta_tile_assign"):
         if k in mangled:
             return k
@@ -776,7 +776,7 @@ def run_op(args, peak, peak_kind):
                   "silu_quant": ["silu_quant_rows"], "router": ["router_topk"],
                   "ep": ["ep_rows", "ep_payload", "ep_combine"],
                   "route_dispatch": ["router_topk", "dispatch_direct", "dispatch_fused", "dispatch_multi",
-                                     "scatter_rows", "scatter_bulk_bf16"]}[args.op]
+                                     "scatter_rows", "scatter_bulk_bf16", "scatter_bulk_fp8"]}[args.op]
     extra["traffic"] = {k: recorded_traffic(k, w.name) for k in op_kernels}
     line = {"op": args.op, "workload": w.name, "us": round(us, 3), "algorithmic_bytes": nbytes,
             "achieved_GBs": round(gbs, 1), "peak": peak, "peak_kind": peak_kind,

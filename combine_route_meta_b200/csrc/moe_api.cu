@@ -81,6 +81,10 @@ int device_info(DeviceInfo **out)
         const size_t big = meta_single_smem(MOE_MAX_EXPERTS);
         if (cudaFuncSetAttribute(meta_single_block, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)big) != cudaSuccess ||
+            cudaFuncSetAttribute(scatter_bulk_fp8<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kBulkMaxSmem) != cudaSuccess ||
+            cudaFuncSetAttribute(scatter_bulk_fp8<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kBulkMaxSmem) != cudaSuccess ||
             cudaFuncSetAttribute(meta_tile_assign, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)meta_assign_smem(MOE_MAX_EXPERTS)) != cudaSuccess ||
             cudaFuncSetAttribute(scatter_bulk_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -398,6 +402,14 @@ int launch_payload(const moe_config *cfg, int32_t T, const void *x, const int32_
         const unsigned grid = grid_for(T, dev->sms, kBulkCtasPerSm);
         const size_t smem = (size_t)kBulkStages * bulk_stage_bytes(cfg->H);
         e = launch(scatter_bulk_bf16, grid, kWarp, smem, s, a);
+    } else if (fp8 && use_bulk_fp8(cfg->H, cfg->k)) {
+        void (*k)(ScatterArgs) = after_layout ? scatter_bulk_fp8<true> : scatter_bulk_fp8<false>;
+        const unsigned block = (unsigned)((cfg->H / 512 + 1) * kWarp); // quantiser warps + store warp
+        const size_t smem = (size_t)kFp8Stages * fp8_stage_bytes(cfg->H);
+        const int per_sm = cached_per_sm((const void *)k, (int)block, smem);
+        if (per_sm == 0)
+            return MOE_ERR_CUDA;
+        e = launch(k, grid_for(T, dev->sms, per_sm), block, smem, s, a);
     } else {
         constexpr int kCols = chunk_cols<kScatterLaneCols>();
         const int64_t warp_units = (int64_t)T * ((cfg->H + kCols - 1) / kCols);

@@ -362,12 +362,134 @@ __global__ void __launch_bounds__(kWarp) scatter_bulk_bf16(ScatterArgs a)
 }
 
 // Whether the bulk scatter applies: bf16 rows of at least 1 KB whose stages fit.
-// fp8 stays on scatter_rows: three bulk-store designs for it (one warp
-// quantising per CTA, CTA-wide staging with a barrier per token, independent
-// warps with per-warp staging) all measured slower than register stores.
 inline bool use_bulk_scatter(int32_t H, bool fp8)
 {
     return !fp8 && H >= 512 && (uint64_t)kBulkStages * bulk_stage_bytes(H) <= kBulkMaxSmem;
+}
+
+// ---- bulk (TMA) scatter, fp8 ------------------------------------------------------
+// The same results as scatter_rows<true>, for rows of 512 to 7680 columns that
+// are whole 512-column chunks and k <= 32.  Register stores fan each warp's
+// 512-byte runs out to k rows at once; whole-row bulk stores keep each
+// destination row one contiguous write, which the HBM write stream favours
+// (the bf16 bulk path reaches 0.98 of the measured copy bandwidth against 0.8
+// for register stores of fp8 codes).
+//
+// One CTA walks tokens t = blockIdx.x, + gridDim.x, ... through a ring of
+// kFp8Stages shared-memory stages (a row's H codes, then its H/128 scales):
+//   - quantiser warps, one per 512-column chunk, load their chunk one token
+//     ahead, quantise it, wait until the stage is free, write the codes and 4
+//     block scales, and arrive on the stage's `full` barrier;
+//   - the store warp waits on `full`, then lane j issues two bulk stores to
+//     slot j (codes, H bytes; scales, H/32 bytes); after committing a token it
+//     waits until the stores issued kFp8Stages - 1 tokens earlier have read
+//     their stage and arrives on that stage's `empty` barrier.
+// The quantisers run up to kFp8Stages tokens ahead of the stores, with no
+// barrier across the CTA.  Every mbarrier wait is bounded (kWaitLimitNs): on
+// expiry the warp sets MOE_DEV_TIMEOUT and leaves the loop, so the others time
+// out too and the CTA ends after draining its bulk stores.
+constexpr int kFp8Stages = 4;
+constexpr int kFp8MaxChunks = 15; // quantiser warps, plus the store warp: at most 512 threads
+
+__host__ __device__ inline uint32_t fp8_stage_bytes(int32_t H) { return (uint32_t)H + (uint32_t)H / 32; }
+
+inline bool use_bulk_fp8(int32_t H, int32_t k)
+{
+    return H % 512 == 0 && H >= 512 && H / 512 <= kFp8MaxChunks && k <= kWarp &&
+           (uint64_t)kFp8Stages * fp8_stage_bytes(H) <= kBulkMaxSmem;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+template <bool kEarlyLoad>
+__global__ void __launch_bounds__((kFp8MaxChunks + 1) * kWarp) scatter_bulk_fp8(ScatterArgs a)
+{
+    constexpr int L = kScatterLaneCols;
+    extern __shared__ __align__(128) uint8_t stage_mem[];
+    __shared__ __align__(8) uint64_t full[kFp8Stages], empty[kFp8Stages];
+    const unsigned lane = lane_id();
+    const int32_t warp = (int32_t)(threadIdx.x / kWarp);
+    const int32_t nq = a.H / 512; // quantiser warps; warp nq stores
+    const uint32_t sb = fp8_stage_bytes(a.H);
+    const int32_t nb = a.H / 128;
+    const int64_t n = ((int64_t)a.T - blockIdx.x + gridDim.x - 1) / gridDim.x;
+    auto token = [&](int64_t i) { return (int32_t)(blockIdx.x + i * gridDim.x); };
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < kFp8Stages; ++st) {
+            mbar_init(smem_addr(&full[st]), (uint32_t)nq);
+            mbar_init(smem_addr(&empty[st]), 1);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp < nq) {
+        LaneData<L> d;
+        if (kEarlyLoad && n > 0)
+            load_chunk<L, true>(a.x + (int64_t)token(0) * a.H, a.H, warp, d);
+        stream_order_begin();
+        if (!kEarlyLoad && n > 0)
+            load_chunk<L, true>(a.x + (int64_t)token(0) * a.H, a.H, warp, d);
+        for (int64_t i = 0; i < n; ++i) {
+            LaneData<L> dn;
+            if (i + 1 < n)
+                load_chunk<L, true>(a.x + (int64_t)token(i + 1) * a.H, a.H, warp, dn);
+            LaneCodes<L> q;
+            quantise_lane<L>(d, q.codes, q.scale);
+            const int st = (int)(i % kFp8Stages);
+            const int64_t use = i / kFp8Stages;
+            if (use > 0 && !mbar_wait(smem_addr(&empty[st]), (uint32_t)((use - 1) & 1), kWaitLimitNs)) {
+                if (lane == 0)
+                    raise_error(a.err, MOE_DEV_TIMEOUT);
+                break;
+            }
+            uint8_t *stage = stage_mem + (uint32_t)st * sb;
+            const int32_t col = warp * 512 + (int32_t)lane * L;
+            *reinterpret_cast<uint4 *>(stage + col) = make_uint4(q.codes[0], q.codes[1], q.codes[2], q.codes[3]);
+            if ((lane & 7) == 0)
+                reinterpret_cast<float *>(stage + a.H)[col / 128] = q.scale;
+            fence_async_shared();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_addr(&full[st]));
+            d = dn;
+        }
+        return;
+    }
+
+    // the store warp
+    stream_order_begin();
+    int32_t my_slot = -1; // lane j holds slot j of the current token
+    if (n > 0 && (int32_t)lane < a.k)
+        my_slot = __ldg(a.slot + (int64_t)token(0) * a.k + lane);
+    for (int64_t i = 0; i < n; ++i) {
+        int32_t next_slot = -1;
+        if (i + 1 < n && (int32_t)lane < a.k)
+            next_slot = __ldg(a.slot + (int64_t)token(i + 1) * a.k + lane);
+        const int st = (int)(i % kFp8Stages);
+        if (!mbar_wait(smem_addr(&full[st]), (uint32_t)((i / kFp8Stages) & 1), kWaitLimitNs)) {
+            if (lane == 0)
+                raise_error(a.err, MOE_DEV_TIMEOUT);
+            break;
+        }
+        const uint8_t *stage = stage_mem + (uint32_t)st * sb;
+        const int32_t s = (int32_t)lane < a.k ? checked_slot(my_slot, a.rows_cap, a.err) : -1;
+        if (s >= 0) {
+            bulk_store(static_cast<uint8_t *>(a.recv_x) + (int64_t)s * a.H, smem_addr(stage), (uint32_t)a.H);
+            bulk_store(a.recv_scale + (int64_t)s * nb, smem_addr(stage + a.H), (uint32_t)nb * 4u);
+        }
+        bulk_commit();
+        // the stores of token i + 1 - kFp8Stages have read their stage: it may be rewritten
+        bulk_wait_read<kFp8Stages - 1>();
+        __syncwarp();
+        if (lane == 0 && i + 1 >= kFp8Stages)
+            mbar_arrive(smem_addr(&empty[(i + 1) % kFp8Stages]));
+        my_slot = next_slot;
+    }
+    bulk_wait_all();
 }
 
 } // namespace moe

@@ -179,6 +179,9 @@ CASES = [
     # narrow bf16 rows with S <= 16384, else metadata kernels + scatter
     (2048, 256, 64, 8, 8, True, True, True),     # S = 16384: the largest mid-size batch
     (2049, 256, 64, 8, 8, True, True, True),     # S = 16392: tiled metadata + fp8 scatter
+    (2050, 7680, 64, 8, 8, True, False, True),   # fp8 bulk scatter, 15 chunk warps per row
+    (2050, 8192, 64, 8, 8, True, False, True),   # one chunk too many: register scatter
+    (700, 1024, 64, 8, 32, True, True, False),   # fp8 bulk scatter, k = 32 slots, duplicates
     (10, 128, 8, 2, 20, False, False, False),
     (600, 1032, 16, 4, 5, False, True, False),   # ragged last 512-column chunk (8 columns)
     (300, 1152, 8, 8, 8, True, True, True),      # 9 scales per row: no 16-byte scale stores
@@ -514,3 +517,26 @@ def test_payload_skips_and_flags_bad_slots(H, fp8):
         for t in (0, 7, T - 1):
             for j in range(k):
                 np.testing.assert_array_equal(got[slot[t, j]].view(np.uint16), x[t])
+
+
+@pytest.mark.parametrize("T,H,E,R,k,fp8,pad128", [
+    (300, 7168, 64, 8, 8, True, False),      # fp8 bulk row stores
+    (257, 512, 32, 4, 6, True, True),        # one chunk warp per row, padding
+    (90, 1152, 16, 4, 4, True, False),       # 9 scales per row: register scatter
+    (300, 2048, 64, 8, 8, False, False),     # bf16 bulk scatter
+])
+def test_layout_then_payload_equals_the_oracle(T, H, E, R, k, fp8, pad128):
+    # the two phases as separate calls (the payload kernels that do not load x
+    # before the previous kernel finishes)
+    x, idx, w = random_problem(T * H, T, H, E, k)
+    cfg = moe.make_config(H, k, E, R, fp8, pad128)
+    buf = moe.Buffers(cfg, T, "cuda")
+    buf.recv_x.view(torch.uint8).fill_(POISON)
+    if buf.recv_scale is not None:
+        buf.recv_scale.view(torch.uint8).fill_(POISON)
+    moe.check()
+    moe.dispatch_layout_into(buf, to_dev(idx))
+    moe.dispatch_payload_into(buf, bf16_to_dev(x))
+    assert moe.check() == 0
+    o = oracle.dispatch(x, idx, E=E, R=R, fp8=fp8, pad128=pad128, rows_cap=buf.rows_cap, recv_fill=POISON)
+    assert_dispatch_equal(dispatch_host(buf), o)
