@@ -208,9 +208,30 @@ class OracleRun:
         return time.perf_counter() - t0
 
 
-def time_oracle(w, budget_s=10.0, max_reps=50):
-    """(GB/s of algorithmic bytes, description) of the oracle on a bounded sample."""
-    run = OracleRun(w)
+class OracleRunParallel(OracleRun):
+    """The same oracle on the same sample, its payload and combine split over
+    every host core by token range (the layout stays one serial walk)."""
+
+    def __init__(self, w, threads):
+        super().__init__(w)
+        self.threads = threads
+        self.desc = (f"oracle dispatch+combine (C, fp64 combine; payload and combine split by "
+                     f"token range over {threads} host threads) on the first {self.ws.T} of "
+                     f"{w.T} tokens of {w.name}")
+
+    def once(self):
+        ws, o = self.ws, self.oracle
+        t0 = time.perf_counter()
+        d = o.dispatch_parallel(self.x, self.idx, E=ws.E, R=ws.R, fp8=ws.fp8, pad128=ws.pad128,
+                                rows_cap=self.cap, threads=self.threads)
+        o.combine_parallel(d["slot"], self.wts, d["recv_x"] if self.eo is None else self.eo, self.threads)
+        return time.perf_counter() - t0
+
+
+def time_oracle(w, budget_s=10.0, max_reps=50, threads=None):
+    """(GB/s of algorithmic bytes, description) of the oracle on a bounded sample
+    (on `threads` host threads when given)."""
+    run = OracleRun(w) if threads is None else OracleRunParallel(w, threads)
     times = []
     t_end = time.perf_counter() + budget_s
     while len(times) < max_reps and (not times or time.perf_counter() < t_end):
@@ -892,6 +913,10 @@ def main():
         g, desc = time_oracle(w0)
         line["cpu_baseline"] = {"value": round(g, 4), "unit": "GB/s", "cores": 1,
                                 "kind": "oracle", "sample": desc}
+        cores = len(os.sched_getaffinity(0))
+        g, desc = time_oracle(w0, budget_s=5.0, threads=cores)
+        line["cpu_baseline_all_cores"] = {"value": round(g, 4), "unit": "GB/s", "cores": cores,
+                                          "kind": "oracle", "sample": desc}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

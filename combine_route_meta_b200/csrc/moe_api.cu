@@ -3,6 +3,7 @@
 // include/moe_dispatch_combine.h.
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include <cuda_runtime.h>
@@ -50,7 +51,7 @@ constexpr int kVersion = 100; // 0.1.0
 
 // Per-device launch facts, read once per device.
 struct DeviceInfo {
-    bool ready = false;
+    std::atomic<bool> ready{false};
     int sms = 0;
     // resident CTAs per SM of the kernels whose grid is one wave
     int silu_per_sm = 1;
@@ -68,6 +69,7 @@ int resident_per_sm(K kernel, int block, size_t smem)
     return n > 0 ? n : 1;
 }
 DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mutex; // the first call on a device fills its entry; later calls read it
 
 int device_info(DeviceInfo **out)
 {
@@ -75,7 +77,12 @@ int device_info(DeviceInfo **out)
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return MOE_ERR_CUDA;
     DeviceInfo &d = g_dev[dev];
-    if (!d.ready) {
+    if (d.ready.load(std::memory_order_acquire)) {
+        *out = &d;
+        return MOE_OK;
+    }
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!d.ready.load(std::memory_order_relaxed)) {
         if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return MOE_ERR_CUDA;
         const size_t big = meta_single_smem(MOE_MAX_EXPERTS);
@@ -100,7 +107,7 @@ int device_info(DeviceInfo **out)
             !(d.send_per_sm[1] = resident_per_sm(combine_partial_send<true>, kPartialThreads, 0)) ||
             !(d.recv_per_sm = resident_per_sm(combine_partial_recv, kPartialThreads, 0)))
             return MOE_ERR_CUDA;
-        d.ready = true;
+        d.ready.store(true, std::memory_order_release);
     }
     *out = &d;
     return MOE_OK;

@@ -333,14 +333,19 @@ __global__ void __launch_bounds__(kWarp) scatter_bulk_bf16(ScatterArgs a)
             bulk_load(smem_addr(stage_mem + s * stage_bytes), a.x + (int64_t)token(i) * a.H, row, bar);
         }
     };
-    for (int64_t i = 0; i < kBulkLookahead && i < n; ++i)
-        issue_load(i);
+    int64_t issued = 0; // loads issued so far: tokens [0, issued)
+    for (; issued < kBulkLookahead && issued < n; ++issued)
+        issue_load(issued);
 
     for (int64_t i = 0; i < n; ++i) {
         const int s = (int)(i % kBulkStages);
         if (!mbar_wait(smem_addr(&bars[s]), (uint32_t)((i / kBulkStages) & 1), kWaitLimitNs)) {
             if (lane == 0)
                 raise_error(a.err, MOE_DEV_TIMEOUT);
+            // drain: the loads issued for tokens [i, issued) may still write
+            // this CTA's shared memory; wait for each, again bounded
+            for (int64_t j = i; j < issued; ++j)
+                mbar_wait(smem_addr(&bars[j % kBulkStages]), (uint32_t)((j / kBulkStages) & 1), kWaitLimitNs);
             break;
         }
         const int32_t t = token(i);
@@ -356,6 +361,7 @@ __global__ void __launch_bounds__(kWarp) scatter_bulk_bf16(ScatterArgs a)
             bulk_wait_read<kBulkStages - kBulkLookahead>();
             __syncwarp();
             issue_load(next);
+            issued = next + 1;
         }
     }
     bulk_wait_all();

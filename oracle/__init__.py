@@ -54,6 +54,10 @@ def _load():
         lib.oracle_dispatch.argtypes = [i32, i32, i32, i32, i32, i32, i32, i64,
                                         P, P, P, P, P, P, P, P, P]
         lib.oracle_dispatch.restype = i32
+        lib.oracle_dispatch_layout.argtypes = [i32, i32, i32, i32, i32, i64, P, P, P, P, P, P]
+        lib.oracle_dispatch_layout.restype = i32
+        lib.oracle_dispatch_payload_rows.argtypes = [i32, i32, i32, i32, i32, P, P, P, P]
+        lib.oracle_dispatch_payload_rows.restype = None
         lib.oracle_combine.argtypes = [i32, i32, i32, P, P, P, P]
         lib.oracle_combine.restype = None
         lib.oracle_combine_rank_partial.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P]
@@ -156,6 +160,60 @@ def dispatch(x_bf16, topk_idx, *, E: int, R: int, fp8: bool, pad128: bool = Fals
     out["err"] = int(err)
     out["rows_cap"] = rows_cap
     return out
+
+
+def _ranges(T: int, parts: int):
+    step = (T + parts - 1) // parts if T else 0
+    return [(a, min(T, a + step)) for a in range(0, T, step)] if step else []
+
+
+def dispatch_parallel(x_bf16, topk_idx, *, E: int, R: int, fp8: bool, pad128: bool = False,
+                      rows_cap: int | None = None, threads: int = 1):
+    """dispatch() with its payload step split over `threads` host threads by
+    token range (the layout stays one serial walk).  The same C functions run on
+    disjoint tokens, so the result is bitwise that of dispatch(); the C calls
+    release the interpreter lock, so the ranges run on separate cores."""
+    from concurrent.futures import ThreadPoolExecutor
+    x = _c(x_bf16, np.uint16)
+    idx = _c(topk_idx, np.int32)
+    T, H = x.shape
+    k = idx.shape[1] if idx.ndim == 2 else 0
+    if rows_cap is None:
+        rows_cap = rows_capacity(T, k, E, pad128)
+    nb = H // 128
+    recv_x = np.zeros((rows_cap, H), np.uint8 if fp8 else np.uint16)
+    recv_scale = np.zeros((rows_cap, nb), np.float32) if fp8 else np.zeros((0, 0), np.float32)
+    out = dict(recv_x=recv_x, recv_scale=recv_scale, expert_count=np.zeros(E, np.int32),
+               expert_offset=np.zeros(E + 1, np.int32), rank_offset=np.zeros(R + 1, np.int32),
+               recv_src=np.zeros(rows_cap, np.int32), slot=np.zeros((T, k), np.int32))
+    lib = _load()
+    out["err"] = int(lib.oracle_dispatch_layout(
+        T, k, E, R, int(bool(pad128)), rows_cap, _ptr(idx), _ptr(out["expert_count"]),
+        _ptr(out["expert_offset"]), _ptr(out["rank_offset"]), _ptr(out["recv_src"]), _ptr(out["slot"])))
+    with ThreadPoolExecutor(max(1, threads)) as ex:
+        list(ex.map(lambda r: lib.oracle_dispatch_payload_rows(
+            r[0], r[1], H, k, int(bool(fp8)), _ptr(x), _ptr(out["slot"]), _ptr(recv_x), _ptr(recv_scale)),
+            _ranges(T, max(1, threads))))
+    out["rows_cap"] = rows_cap
+    return out
+
+
+def combine_parallel(slot, topk_w, expert_out_bf16, threads: int = 1) -> np.ndarray:
+    """combine() over `threads` host threads by token range; bitwise the same."""
+    from concurrent.futures import ThreadPoolExecutor
+    slot = _c(slot, np.int32)
+    w = _c(topk_w, np.float32)
+    eo = _c(expert_out_bf16, np.uint16)
+    T = slot.shape[0]
+    k = slot.shape[1] if slot.ndim == 2 else 0
+    H = eo.shape[1]
+    y = np.zeros((T, H), np.float64)
+    lib = _load()
+    with ThreadPoolExecutor(max(1, threads)) as ex:
+        list(ex.map(lambda r: lib.oracle_combine(r[1] - r[0], H, k, _ptr(slot[r[0]:r[1]]), _ptr(w[r[0]:r[1]]),
+                                                 _ptr(eo), _ptr(y[r[0]:r[1]])),
+                    _ranges(T, max(1, threads))))
+    return y
 
 
 def combine(slot, topk_w, expert_out_bf16, tokens=None) -> np.ndarray:

@@ -143,12 +143,14 @@ static int64_t padded(int64_t count, int32_t pad128)
  *   with recv_scale[slot, H/128]) for every kept entry.
  * Returns the OR of the error bits.
  */
-int32_t oracle_dispatch(int32_t T, int32_t H, int32_t k, int32_t E, int32_t R,
-                        int32_t fp8, int32_t pad128, int64_t rows_cap,
-                        const uint16_t *x, const int32_t *topk_idx,
-                        void *recv_x, float *recv_scale,
-                        int32_t *expert_count, int32_t *expert_offset,
-                        int32_t *rank_offset, int32_t *recv_src, int32_t *slot)
+/*
+ * Steps 1-4 of the dispatch (counts, offsets, rank offsets, slots and
+ * recv_src); returns the error bits.
+ */
+int32_t oracle_dispatch_layout(int32_t T, int32_t k, int32_t E, int32_t R, int32_t pad128,
+                               int64_t rows_cap, const int32_t *topk_idx,
+                               int32_t *expert_count, int32_t *expert_offset,
+                               int32_t *rank_offset, int32_t *recv_src, int32_t *slot)
 {
     int32_t err = 0;
 
@@ -199,16 +201,25 @@ int32_t oracle_dispatch(int32_t T, int32_t H, int32_t k, int32_t E, int32_t R,
             recv_src[s] = (int32_t)i;
         }
     free(cursor);
+    return err;
+}
 
-    /* 5. Payload: the token's row (or its e4m3 codes and scales) to every slot. */
+/*
+ * Step 5 of the dispatch for tokens [t0, t1): the token's row (or its e4m3
+ * codes and scales) to every slot.
+ */
+void oracle_dispatch_payload_rows(int32_t t0, int32_t t1, int32_t H, int32_t k, int32_t fp8,
+                                  const uint16_t *x, const int32_t *slot, void *recv_x,
+                                  float *recv_scale)
+{
     int32_t nb = H / 128;
     uint8_t *codes = NULL;
     float *scales = NULL;
     if (fp8) {
-        codes = (uint8_t *)malloc((size_t)H);
+        codes = (uint8_t *)malloc((size_t)(H > 0 ? H : 1));
         scales = (float *)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
     }
-    for (int32_t t = 0; t < T; ++t) {
+    for (int32_t t = t0; t < t1; ++t) {
         const uint16_t *xt = x + (int64_t)t * H;
         if (fp8)
             quantise_row_fp8(xt, H, codes, scales);
@@ -226,6 +237,18 @@ int32_t oracle_dispatch(int32_t T, int32_t H, int32_t k, int32_t E, int32_t R,
     }
     free(codes);
     free(scales);
+}
+
+int32_t oracle_dispatch(int32_t T, int32_t H, int32_t k, int32_t E, int32_t R,
+                        int32_t fp8, int32_t pad128, int64_t rows_cap,
+                        const uint16_t *x, const int32_t *topk_idx,
+                        void *recv_x, float *recv_scale,
+                        int32_t *expert_count, int32_t *expert_offset,
+                        int32_t *rank_offset, int32_t *recv_src, int32_t *slot)
+{
+    const int32_t err = oracle_dispatch_layout(T, k, E, R, pad128, rows_cap, topk_idx, expert_count,
+                                               expert_offset, rank_offset, recv_src, slot);
+    oracle_dispatch_payload_rows(0, T, H, k, fp8, x, slot, recv_x, recv_scale);
     return err;
 }
 

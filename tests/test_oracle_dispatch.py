@@ -207,3 +207,17 @@ def test_workload_table_shapes():
         assert w.E % w.R == 0
         if w.fp8:
             assert w.H % 128 == 0
+
+
+@pytest.mark.parametrize("fp8,pad128,threads", [(True, True, 4), (False, False, 3), (True, False, 8)])
+def test_parallel_runner_is_bitwise_the_serial_oracle(fp8, pad128, threads):
+    # the host-thread split used for the all-cores CPU baseline changes nothing
+    from workloads import random_problem
+    x, idx, w = random_problem(21, 301, 256, 16, 4)
+    a = oracle.dispatch(x, idx, E=16, R=4, fp8=fp8, pad128=pad128)
+    b = oracle.dispatch_parallel(x, idx, E=16, R=4, fp8=fp8, pad128=pad128, threads=threads)
+    for key in ("recv_x", "recv_scale", "expert_count", "expert_offset", "rank_offset", "recv_src", "slot"):
+        np.testing.assert_array_equal(a[key], b[key], err_msg=key)
+    assert a["err"] == b["err"]
+    eo = a["recv_x"] if not fp8 else np.resize(x, (a["rows_cap"], 256))
+    np.testing.assert_array_equal(oracle.combine(a["slot"], w, eo), oracle.combine_parallel(a["slot"], w, eo, threads))
