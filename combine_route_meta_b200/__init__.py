@@ -452,8 +452,8 @@ def route_dispatch_into(buf: Buffers, x: torch.Tensor, logits: torch.Tensor, top
                         topk_w: torch.Tensor, *, score_fn: str = "softmax", n_group: int = 1,
                         topk_group: int = 1, renormalize: bool = True,
                         stream: Optional[torch.cuda.Stream] = None) -> None:
-    """moe_route_dispatch into preallocated buffers: the router writes topk_idx
-    and topk_w, then the dispatch reads them."""
+    """moe_route_dispatch into preallocated buffers: the routing writes topk_idx
+    and topk_w and the dispatch reads them (one launch at decode sizes)."""
     P = ctypes.c_void_p
     st = lib.moe_route_dispatch(ctypes.byref(buf.cfg), buf.T, P(x.data_ptr()), P(logits.data_ptr()),
                                 {"softmax": SCORE_SOFTMAX, "sigmoid": SCORE_SIGMOID}[score_fn],

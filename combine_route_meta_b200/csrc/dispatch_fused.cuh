@@ -23,6 +23,7 @@
 
 #include "common.cuh"
 #include "meta.cuh"
+#include "router.cuh"
 #include "scatter.cuh"
 
 namespace moe {
@@ -171,62 +172,100 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_fused(FusedArgs 
 // finish them, so no per-expert histogram or scan sits on the token's path.
 // One extra CTA (blockIdx.x == T) writes the per-expert counts and offsets, the
 // rank offsets and the unused rows' recv_src, and flags bad expert ids.
-template <int kChunks, bool kFp8, int kK>
-__global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct(FusedArgs a)
+// An expert id: from global memory through the read-only path (dispatch_direct,
+// whose ids another kernel wrote), or from this CTA's shared memory (the fused
+// router, which routes every token into it).
+template <bool kShared>
+__device__ __forceinline__ int32_t load_id(const int32_t *p)
 {
-    stream_order_begin();
-    extern __shared__ int32_t sm[];
-    __shared__ uint32_t s_part[kFusedMaxThreads / kWarp][kK];
-    __shared__ int32_t s_slot[kK];
-    __shared__ int32_t s_own[kK];
+    if constexpr (kShared)
+        return *p;
+    else
+        return __ldg(p);
+}
 
-    const int32_t t = blockIdx.x;
+// The metadata CTA of the direct-rank dispatch: histogram, scan, offsets, and
+// recv_src = -1 past the last segment (without padding there are no gaps
+// between segments).  It runs beside the token CTAs and is about as long, so
+// it is kept lean.  sm: E + 1 + E int32 of shared memory.
+template <bool kIdsShared>
+__device__ __forceinline__ void direct_meta_cta(const FusedArgs &a, const int32_t *ids, int32_t *sm)
+{
+    const int nt = blockDim.x;
+    const int64_t S = (int64_t)a.T * a.k;
+    int32_t *hist = sm, *off = sm + a.E;
+    for (int32_t e = threadIdx.x; e < a.E; e += nt)
+        hist[e] = 0;
+    __syncthreads();
+    const int32_t S32 = (int32_t)S; // S <= kFusedMaxEntries
+    for (int32_t base = 0; base < S32; base += nt * kFusedLoadRounds) {
+        int32_t ev[kFusedLoadRounds];
+#pragma unroll
+        for (int r = 0; r < kFusedLoadRounds; ++r) {
+            const int32_t i = base + r * nt + (int32_t)threadIdx.x;
+            ev[r] = i < S32 ? load_id<kIdsShared>(ids + i) : 0;
+        }
+#pragma unroll
+        for (int r = 0; r < kFusedLoadRounds; ++r) {
+            if (base + r * nt + (int32_t)threadIdx.x >= S32)
+                break;
+            if ((uint32_t)ev[r] < (uint32_t)a.E)
+                atomicAdd(&hist[ev[r]], 1);
+            else
+                raise_error(a.err, MOE_DEV_BAD_INDEX);
+        }
+    }
+    __syncthreads();
+    block_offsets(hist, off, a.E, 0);
+    for (int32_t e = threadIdx.x; e < a.E; e += nt) {
+        a.expert_count[e] = hist[e];
+        a.expert_offset[e] = off[e];
+    }
+    if (threadIdx.x == 0)
+        a.expert_offset[a.E] = off[a.E];
+    for (int32_t r = threadIdx.x; r <= a.R; r += nt)
+        a.rank_offset[r] = off[r * (a.E / a.R)];
+    block_fill_tail(a.rows_cap, a.E, a.recv_src, off, 0, 1);
+}
+
+// Loads the token's row: warp w owns chunks w, w + nwarps, ...
+template <int kChunks, bool kFp8>
+__device__ __forceinline__ void direct_load_row(const FusedArgs &a, int32_t t, LaneData<kFusedLaneCols> (&d)[kChunks])
+{
+    constexpr int L = kFusedLaneCols;
+    const int nwarps = blockDim.x / kWarp;
+    const int warp = threadIdx.x / kWarp;
+    const int32_t chunks = (a.H + chunk_cols<L>() - 1) / chunk_cols<L>();
+    const uint16_t *xr = a.x + (int64_t)t * a.H;
+#pragma unroll
+    for (int i = 0; i < kChunks; ++i) {
+        const int32_t c = warp + i * nwarps;
+        if (c < chunks)
+            load_chunk<L, kFp8>(xr, a.H, c, d[i]);
+    }
+}
+
+// Shared memory of a direct-rank token CTA.
+template <int kK>
+struct DirectShared {
+    uint32_t part[kFusedMaxThreads / kWarp][kK];
+    int32_t slot[kK];
+    int32_t own[kK];
+};
+
+// A token CTA of the direct-rank dispatch, from the expert ids on; with
+// kRowLoaded the row is already in d (else it is loaded after the ids go out).
+template <int kChunks, bool kFp8, int kK, bool kRowLoaded, bool kIdsShared>
+__device__ __forceinline__ void direct_token_cta(const FusedArgs &a, const int32_t *ids, int32_t t,
+                                                 LaneData<kFusedLaneCols> (&d)[kChunks],
+                                                 LaneCodes<kFusedLaneCols> (&q)[kFp8 ? kChunks : 1],
+                                                 bool quantised, DirectShared<kK> &sh)
+{
     const int nt = blockDim.x;
     const int nwarps = nt / kWarp;
     const int warp = threadIdx.x / kWarp;
     const unsigned lane = lane_id();
     const int64_t S = (int64_t)a.T * a.k;
-
-    if (t == a.T) {
-        // metadata CTA: histogram, scan, offsets, and recv_src = -1 past the
-        // last segment (without padding there are no gaps between segments).
-        // It runs beside the token CTAs and is about as long, so it is kept lean.
-        int32_t *hist = sm, *off = sm + a.E;
-        for (int32_t e = threadIdx.x; e < a.E; e += nt)
-            hist[e] = 0;
-        __syncthreads();
-        const int32_t S32 = (int32_t)S; // S <= kFusedMaxEntries
-        for (int32_t base = 0; base < S32; base += nt * kFusedLoadRounds) {
-            int32_t ev[kFusedLoadRounds];
-#pragma unroll
-            for (int r = 0; r < kFusedLoadRounds; ++r) {
-                const int32_t i = base + r * nt + (int32_t)threadIdx.x;
-                ev[r] = i < S32 ? __ldg(a.topk_idx + i) : 0;
-            }
-#pragma unroll
-            for (int r = 0; r < kFusedLoadRounds; ++r) {
-                if (base + r * nt + (int32_t)threadIdx.x >= S32)
-                    break;
-                if ((uint32_t)ev[r] < (uint32_t)a.E)
-                    atomicAdd(&hist[ev[r]], 1);
-                else
-                    raise_error(a.err, MOE_DEV_BAD_INDEX);
-            }
-        }
-        __syncthreads();
-        block_offsets(hist, off, a.E, 0);
-        for (int32_t e = threadIdx.x; e < a.E; e += nt) {
-            a.expert_count[e] = hist[e];
-            a.expert_offset[e] = off[e];
-        }
-        if (threadIdx.x == 0)
-            a.expert_offset[a.E] = off[a.E];
-        for (int32_t r = threadIdx.x; r <= a.R; r += nt)
-            a.rank_offset[r] = off[r * (a.E / a.R)];
-        block_fill_tail(a.rows_cap, a.E, a.recv_src, off, 0, 1);
-        return;
-    }
-
     constexpr int L = kFusedLaneCols;
     const int32_t chunks = (a.H + chunk_cols<L>() - 1) / chunk_cols<L>();
     const int64_t mine = (int64_t)t * a.k;
@@ -241,7 +280,7 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct(FusedArgs
     if constexpr (kOwnInRegs) {
 #pragma unroll
         for (int j = 0; j < kK; ++j) {
-            const int32_t e = j < a.k ? __ldg(a.topk_idx + mine + j) : -1;
+            const int32_t e = j < a.k ? load_id<kIdsShared>(ids + mine + j) : -1;
             own[j] = (uint32_t)e < (uint32_t)a.E ? e : -1;
         }
     }
@@ -249,21 +288,15 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct(FusedArgs
 #pragma unroll
     for (int r = 0; r < kFusedLoadRounds; ++r) {
         const int32_t i = r * nt + (int32_t)threadIdx.x;
-        ev[r] = i < S32 ? __ldg(a.topk_idx + i) : kNone;
+        ev[r] = i < S32 ? load_id<kIdsShared>(ids + i) : kNone;
     }
 
     // 2. The row: warp w owns chunks w, w + nwarps, ...
-    const uint16_t *xr = a.x + (int64_t)t * a.H;
-    LaneData<L> d[kChunks];
-#pragma unroll
-    for (int i = 0; i < kChunks; ++i) {
-        const int32_t c = warp + i * nwarps;
-        if (c < chunks)
-            load_chunk<L, kFp8>(xr, a.H, c, d[i]);
-    }
+    if constexpr (!kRowLoaded)
+        direct_load_row<kChunks, kFp8>(a, t, d);
     if ((int)threadIdx.x < kK) {
-        const int32_t e = (int)threadIdx.x < a.k ? __ldg(a.topk_idx + mine + threadIdx.x) : -1;
-        s_own[threadIdx.x] = (e >= 0 && e < a.E) ? e : -1;
+        const int32_t e = (int)threadIdx.x < a.k ? load_id<kIdsShared>(ids + mine + threadIdx.x) : -1;
+        sh.own[threadIdx.x] = (e >= 0 && e < a.E) ? e : -1;
     }
     if constexpr (!kOwnInRegs)
         __syncthreads();
@@ -279,7 +312,7 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct(FusedArgs
 #pragma unroll
             for (int r = 0; r < kFusedLoadRounds; ++r) {
                 const int32_t i = base + r * nt + (int32_t)threadIdx.x;
-                ev[r] = i < S32 ? __ldg(a.topk_idx + i) : kNone;
+                ev[r] = i < S32 ? load_id<kIdsShared>(ids + i) : kNone;
             }
         }
 #pragma unroll
@@ -293,7 +326,7 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct(FusedArgs
             const int32_t before = i - mine32; // entry i precedes (t, j) when before < j
 #pragma unroll
             for (int j = 0; j < kK; ++j) {
-                const uint32_t o = (uint32_t)(kOwnInRegs ? own[kOwnInRegs ? j : 0] : s_own[j]);
+                const uint32_t o = (uint32_t)(kOwnInRegs ? own[kOwnInRegs ? j : 0] : sh.own[j]);
                 cnt[j] += e < o ? 1u : 0u;
                 cnt[j] += (e == o && before < j) ? 0x10000u : 0u;
             }
@@ -303,17 +336,17 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct(FusedArgs
     for (int j = 0; j < kK; ++j) {
         const uint32_t w = __reduce_add_sync(kFullMask, cnt[j]);
         if (lane == 0)
-            s_part[warp][j] = w;
+            sh.part[warp][j] = w;
     }
     __syncthreads();
 
     // 4. This token's slots: warp j adds the per-warp counts of entry j.
     for (int j = warp; j < a.k; j += nwarps) {
-        const uint32_t v = (int)lane < nwarps ? s_part[lane][j] : 0u;
+        const uint32_t v = (int)lane < nwarps ? sh.part[lane][j] : 0u;
         const uint32_t tot = __reduce_add_sync(kFullMask, v);
         if (lane == 0) {
             int32_t s = -1;
-            if (s_own[j] >= 0) {
+            if (sh.own[j] >= 0) {
                 const int64_t row = (int64_t)(tot & 0xffffu) + (tot >> 16);
                 if (row < a.rows_cap) {
                     s = (int32_t)row;
@@ -323,17 +356,18 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct(FusedArgs
                 }
             }
             a.slot[mine + j] = s;
-            s_slot[j] = s;
+            sh.slot[j] = s;
         }
     }
 
-    // 5. The row's codes, while the slot sums above complete.
-    LaneCodes<L> q[kFp8 ? kChunks : 1];
+    // 5. The row's codes (unless already made), while the slot sums above complete.
     if constexpr (kFp8) {
+        if (!quantised) {
 #pragma unroll
-        for (int i = 0; i < kChunks; ++i)
-            if (warp + i * nwarps < chunks)
-                quantise_lane<L>(d[i], q[i].codes, q[i].scale);
+            for (int i = 0; i < kChunks; ++i)
+                if (warp + i * nwarps < chunks)
+                    quantise_lane<L>(d[i], q[i].codes, q[i].scale);
+        }
     }
     __syncthreads();
 
@@ -344,10 +378,62 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct(FusedArgs
         if (c >= chunks)
             continue;
         if constexpr (kFp8)
-            store_codes<L>(a.recv_x, a.recv_scale, a.H, c, a.k, s_slot, a.rows_cap, a.err, q[i]);
+            store_codes<L>(a.recv_x, a.recv_scale, a.H, c, a.k, sh.slot, a.rows_cap, a.err, q[i]);
         else
-            store_chunk<L, false>(a.recv_x, a.recv_scale, a.H, c, a.k, s_slot, a.rows_cap, a.err, d[i]);
+            store_chunk<L, false>(a.recv_x, a.recv_scale, a.H, c, a.k, sh.slot, a.rows_cap, a.err, d[i]);
     }
+}
+
+template <int kChunks, bool kFp8, int kK>
+__global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct(FusedArgs a)
+{
+    stream_order_begin();
+    extern __shared__ int32_t sm[];
+    __shared__ DirectShared<kK> sh;
+    const int32_t t = blockIdx.x;
+    if (t == a.T) {
+        direct_meta_cta<false>(a, a.topk_idx, sm);
+        return;
+    }
+    LaneData<kFusedLaneCols> d[kChunks];
+    LaneCodes<kFusedLaneCols> q[kFp8 ? kChunks : 1];
+    direct_token_cta<kChunks, kFp8, kK, false, false>(a, a.topk_idx, t, d, q, false, sh);
+}
+
+// ---- after the router (decode) ----------------------------------------------------
+// dispatch_direct for moe_route_dispatch, launched right after the router in
+// the same stream.  The row of x and (fp8) its codes do not depend on the
+// routing, and the router writes neither x nor anything x depends on; it
+// waited for every earlier kernel before it let this one launch, so x is
+// complete when this kernel starts.  Each token CTA therefore loads and
+// quantises its row while the router is still running, and waits for the
+// router (griddepcontrol.wait) only before it reads the expert ids.  (The x
+// loads do not allocate in L1, so no stale line can exist.)
+template <int kChunks, bool kFp8, int kK>
+__global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct_after_router(FusedArgs a)
+{
+    extern __shared__ int32_t sm[];
+    __shared__ DirectShared<kK> sh;
+    const int32_t t = blockIdx.x;
+    LaneData<kFusedLaneCols> d[kChunks];
+    LaneCodes<kFusedLaneCols> q[kFp8 ? kChunks : 1];
+    if (t < a.T) {
+        direct_load_row<kChunks, kFp8>(a, t, d);
+        if constexpr (kFp8) {
+            const int nwarps = blockDim.x / kWarp, warp = threadIdx.x / kWarp;
+            const int32_t chunks = (a.H + chunk_cols<kFusedLaneCols>() - 1) / chunk_cols<kFusedLaneCols>();
+#pragma unroll
+            for (int i = 0; i < kChunks; ++i)
+                if (warp + i * nwarps < chunks)
+                    quantise_lane<kFusedLaneCols>(d[i], q[i].codes, q[i].scale);
+        }
+    }
+    stream_order_begin();
+    if (t == a.T) {
+        direct_meta_cta<false>(a, a.topk_idx, sm);
+        return;
+    }
+    direct_token_cta<kChunks, kFp8, kK, true, false>(a, a.topk_idx, t, d, q, kFp8, sh);
 }
 
 } // namespace moe

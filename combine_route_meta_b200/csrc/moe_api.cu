@@ -253,12 +253,23 @@ int cached_per_sm(const void *fn, int block, size_t smem)
 // fewest that fit the row in one CTA).  It runs only for T below the SM count
 // (larger small batches take dispatch_multi), so its T (+1) CTAs of at most
 // 1024 threads are resident in one wave.
-cudaError_t launch_small(bool fp8, int per, int32_t T, cudaStream_t s, const FusedArgs &f)
+// after_router: the previous kernel in the stream is the router of the same
+// moe_route_dispatch call, so the direct-rank kernel may load x before waiting.
+cudaError_t launch_small(bool fp8, int per, int32_t T, cudaStream_t s, const FusedArgs &f, bool after_router)
 {
     const bool pad = f.pad128 != 0;
     const unsigned grid = pad ? (unsigned)T : (unsigned)T + 1;
     const int32_t chunks = (f.H + chunk_cols<kFusedLaneCols>() - 1) / chunk_cols<kFusedLaneCols>();
     const unsigned block = (unsigned)((chunks + per - 1) / per * kWarp);
+    if (after_router && !pad && f.k <= 8) {
+        const int i = per == 1 ? 0 : (per == 2 ? 1 : 2);
+        static const SmallKernel t[2][3] = {
+            {dispatch_direct_after_router<1, false, 8>, dispatch_direct_after_router<2, false, 8>,
+             dispatch_direct_after_router<4, false, 8>},
+            {dispatch_direct_after_router<1, true, 8>, dispatch_direct_after_router<2, true, 8>,
+             dispatch_direct_after_router<4, true, 8>}};
+        return launch(t[fp8][i], grid, block, fused_smem(f.E), s, f);
+    }
     return launch(small_kernel(fp8, pad, f.k > 8, per), grid, block, fused_smem(f.E), s, f);
 }
 
@@ -565,7 +576,7 @@ int launch_router(int32_t T, int32_t E, int32_t k, const float *logits, int32_t 
 int run_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t *topk_idx,
                  const float *topk_w, const moe_dispatch_out *out, int32_t *slot,
                  void *workspace, int32_t *dev_err, DeviceInfo *dev, cudaStream_t s,
-                 moe_handle *handle);
+                 moe_handle *handle, bool after_router = false);
 
 } // namespace
 
@@ -584,6 +595,10 @@ int moe_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
     return run_dispatch(cfg, T, x, topk_idx, topk_w, out, slot, workspace, dev_err, dev,
                         static_cast<cudaStream_t>(stream), handle);
 }
+
+namespace {
+
+} // namespace
 
 int moe_route_dispatch(const moe_config *cfg, int32_t T, const void *x, const float *logits,
                        int32_t score_fn, int32_t n_group, int32_t topk_group, int32_t renormalize,
@@ -606,7 +621,8 @@ int moe_route_dispatch(const moe_config *cfg, int32_t T, const void *x, const fl
     if (T > 0 && (st = launch_router(T, cfg->E, cfg->k, logits, score_fn, n_group, topk_group,
                                      renormalize, topk_idx, topk_w, dev, s)) != MOE_OK)
         return st;
-    return run_dispatch(cfg, T, x, topk_idx, topk_w, out, slot, workspace, dev_err, dev, s, handle);
+    return run_dispatch(cfg, T, x, topk_idx, topk_w, out, slot, workspace, dev_err, dev, s, handle,
+                        true);
 }
 
 namespace {
@@ -614,7 +630,7 @@ namespace {
 int run_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t *topk_idx,
                  const float *topk_w, const moe_dispatch_out *out, int32_t *slot,
                  void *workspace, int32_t *dev_err, DeviceInfo *dev, cudaStream_t s,
-                 moe_handle *handle)
+                 moe_handle *handle, bool after_router)
 {
     int st;
     const bool fp8 = cfg->flags & MOE_FP8;
@@ -639,7 +655,7 @@ int run_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
         f.recv_src = out->recv_src;
         f.slot = slot;
         f.err = dev_err;
-        const cudaError_t e = launch_small(fp8, per, T, s, f);
+        const cudaError_t e = launch_small(fp8, per, T, s, f, after_router);
         if ((st = launched(e)) != MOE_OK)
             return st;
     } else if (use_multi(cfg, T)) {

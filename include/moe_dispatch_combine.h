@@ -327,15 +327,20 @@ MOE_API int moe_router_topk(int32_t T, int32_t E, int32_t k, const float *logits
                             int32_t renormalize, int32_t *topk_idx, float *topk_w, void *stream);
 
 /*
- * Router top-k followed by dispatch, in one call: moe_router_topk on logits[T,
- * E] (E = cfg->E, k = cfg->k) writes topk_idx[T, k] and topk_w[T, k], and
- * moe_dispatch then reads them ("Lower latency and higher throughput with
- * multi-node DeepSeek deployment", section "Roteador MoE": the router is the
- * step right before dispatch).  The two kernels are stream-ordered and the
- * second starts launching while the first finishes; the ids and weights
- * (a few KB at decode sizes) are read back from L2.  Every argument of both
- * steps is checked before anything is enqueued; results, errors and the
- * handle are those of the two calls made one after the other.
+ * Router top-k followed by dispatch, in one call: the routing of moe_router_topk
+ * on logits[T, E] (E = cfg->E, k = cfg->k) writes topk_idx[T, k] and
+ * topk_w[T, k], and the dispatch of moe_dispatch reads them ("Lower latency and
+ * higher throughput with multi-node DeepSeek deployment", section "Roteador
+ * MoE": the router is the step right before dispatch).  Results, errors and
+ * the handle are those of the two calls made one after the other.
+ *
+ * The router and the dispatch are two stream-ordered launches.  At decode
+ * sizes (no MOE_PAD128, k <= 8, T below the SM count: the one-token-per-CTA
+ * dispatch) the dispatch kernel starts while the router runs and loads and
+ * quantises its rows before it waits for the router, so only the work that
+ * needs the expert ids (a few KB, read from L2) follows the router.
+ * workspace is moe_dispatch's (moe_workspace_bytes(cfg, T)).  Every argument
+ * of both steps is checked before anything is enqueued.
  */
 MOE_API int moe_route_dispatch(const moe_config *cfg, int32_t T, const void *x,
                                const float *logits, int32_t score_fn, int32_t n_group,

@@ -247,8 +247,14 @@ def test_router_topk_ties_zeros_and_infinities(E, G, TG, fn):
 # ---- router feeding dispatch in one call ------------------------------------------------
 
 @pytest.mark.parametrize("T,E,R,k,H,fn,G,TG,fp8,pad", [
-    (128, 256, 8, 8, 7168, "sigmoid", 8, 4, True, False),   # DeepSeek-V3-shaped decode
+    (128, 256, 8, 8, 7168, "sigmoid", 8, 4, True, False),   # DeepSeek-V3-shaped decode (one launch)
+    (128, 384, 16, 8, 7168, "softmax", 1, 1, True, False),  # Kimi-K2-shaped: 12 logits per lane
     (16, 8, 2, 2, 256, "softmax", 1, 1, False, False),
+    (1, 64, 4, 4, 1024, "sigmoid", 4, 2, False, False),     # one token
+    (147, 256, 8, 8, 2048, "softmax", 1, 1, True, False),   # 148 CTAs: every SM
+    (20, 128, 8, 6, 16384, "sigmoid", 1, 1, True, False),   # 2 chunks per warp
+    (9, 32, 4, 8, 24576, "softmax", 1, 1, False, False),    # 4 chunks per warp
+    (64, 256, 8, 8, 7168, "softmax", 1, 1, True, True),     # padding: router, then dispatch
     (3000, 256, 32, 8, 512, "softmax", 1, 1, True, True),   # tiled metadata path
 ])
 def test_route_dispatch_equals_router_then_dispatch(T, E, R, k, H, fn, G, TG, fp8, pad):
@@ -272,3 +278,51 @@ def test_route_dispatch_equals_router_then_dispatch(T, E, R, k, H, fn, G, TG, fp
                                   d2.recv_x[:n][valid].view(torch.uint8).cpu().numpy())
     o = oracle.dispatch(x, ref_idx, E=E, R=R, fp8=fp8, pad128=pad)
     np.testing.assert_array_equal(d.handle.slot.cpu().numpy(), o["slot"])
+
+
+def _graph_kernel_count(fn):
+    """Kernel nodes of a CUDA graph captured around fn() (after one warm-up call)."""
+    from cuda.bindings import driver as drv
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph(keep_graph=True)
+    with torch.cuda.graph(g):
+        fn()
+    graph = drv.CUgraph(g.raw_cuda_graph())
+    _, _, n = drv.cuGraphGetNodes(graph, 0)
+    _, nodes, n = drv.cuGraphGetNodes(graph, n)
+    kinds = [drv.cuGraphNodeGetType(node)[1] for node in nodes[:n]]
+    return sum(k == drv.CUgraphNodeType.CU_GRAPH_NODE_TYPE_KERNEL for k in kinds)
+
+
+def test_route_dispatch_repeats_on_the_same_buffers():
+    # the dispatch kernel after the router reads x before the router has
+    # finished: fresh logits each call must still give the oracle's choice and
+    # dispatch, call after call and in a captured graph
+    T, E, R, k, H = 128, 256, 8, 8, 7168
+    rng = np.random.default_rng(41)
+    xh = f32_to_bf16_bits(rng.standard_normal((T, H)).astype(np.float32))
+    x = bf16_to_dev(xh)
+    cfg = moe.make_config(H, k, E, R, True, False)
+    buf = moe.Buffers(cfg, T, "cuda")
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    wt = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    moe.check()
+    for rep in range(3):
+        logits = rng.standard_normal((T, E)).astype(np.float32)
+        moe.route_dispatch_into(buf, x, to_dev(logits), idx, wt, score_fn="sigmoid")
+        torch.cuda.synchronize()
+        assert moe.check() == 0
+        ref_idx, _ = oracle.router_topk(logits, k, score_fn="sigmoid")
+        np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
+        o = oracle.dispatch(xh, ref_idx, E=E, R=R, fp8=True, rows_cap=buf.rows_cap)
+        np.testing.assert_array_equal(buf.slot.cpu().numpy(), o["slot"])
+        valid = o["recv_src"] >= 0
+        np.testing.assert_array_equal(buf.recv_x.view(torch.uint8).cpu().numpy()[valid], o["recv_x"][valid])
+    ld = to_dev(rng.standard_normal((T, E)).astype(np.float32))
+    assert _graph_kernel_count(lambda: moe.route_dispatch_into(buf, x, ld, idx, wt, score_fn="sigmoid")) == 2
+    assert moe.check() == 0
