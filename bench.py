@@ -313,6 +313,7 @@ def config_for(w, world, rows_cap):
             "l2": ("inputs larger than 2x L2 every step (no flush needed)" if one_set else
                    "rotating input sets: over 2x L2 of other sets touched between uses of a set"),
             "graphs": "CUDA graphs of 8+ steps over the rotating sets, replayed back to back",
+            "inputs": "written before the step; the dispatch is told so (MOE_INPUTS_READY)",
             "parallelism": f"replicas x{world}"}
 
 
@@ -330,7 +331,10 @@ def run_gpu(args, name, rank, world, with_e2e):
     if w.identity_experts and w.fp8:
         raise SystemExit("identity experts need a bf16 dispatch")
     _, x, idx, wts = make_inputs(w)
-    cfg = moe.make_config(w.H, w.k, w.E, w.R, w.fp8, w.pad128)
+    # Every step's inputs were written before the kernel ahead of its dispatch
+    # (that kernel is the previous step's combine, or in the end-to-end loop the
+    # inputs arrive by host copies): MOE_INPUTS_READY holds.
+    cfg = moe.make_config(w.H, w.k, w.E, w.R, w.fp8, w.pad128, inputs_ready=True)
     rows_cap = moe.rows_capacity(cfg, w.T)
     eo_host = None if w.identity_experts else make_expert_out(w, rows_cap)
 

@@ -36,6 +36,7 @@ if not os.path.exists(LIB_PATH):
 
 FP8 = 1
 PAD128 = 2
+INPUTS_READY = 4
 
 OK = 0
 ERR_INVALID_ARG = -1
@@ -175,9 +176,10 @@ def _ok(status: int, what: str):
 # ---- torch-level helpers ------------------------------------------------------
 
 def make_config(H: int, k: int, num_experts: int, num_virtual_ranks: int,
-                fp8: bool, pad128: bool = False) -> moe_config:
+                fp8: bool, pad128: bool = False, inputs_ready: bool = False) -> moe_config:
+    """inputs_ready: MOE_INPUTS_READY (see the C header)."""
     return moe_config(H, k, num_experts, num_virtual_ranks,
-                      (FP8 if fp8 else 0) | (PAD128 if pad128 else 0))
+                      (FP8 if fp8 else 0) | (PAD128 if pad128 else 0) | (INPUTS_READY if inputs_ready else 0))
 
 
 def rows_capacity(cfg: moe_config, T: int) -> int:

@@ -188,9 +188,12 @@ __device__ __forceinline__ int32_t load_id(const int32_t *p)
 // recv_src = -1 past the last segment (without padding there are no gaps
 // between segments).  It runs beside the token CTAs and is about as long, so
 // it is kept lean.  sm: E + 1 + E int32 of shared memory.
-template <bool kIdsShared>
+// With kDeferWrites the CTA reads and computes before waiting for the
+// previous kernel in the stream (stream_order_begin) and writes only after it.
+template <bool kIdsShared, bool kDeferWrites = false>
 __device__ __forceinline__ void direct_meta_cta(const FusedArgs &a, const int32_t *ids, int32_t *sm)
 {
+    bool bad = false;
     const int nt = blockDim.x;
     const int64_t S = (int64_t)a.T * a.k;
     int32_t *hist = sm, *off = sm + a.E;
@@ -212,11 +215,15 @@ __device__ __forceinline__ void direct_meta_cta(const FusedArgs &a, const int32_
             if ((uint32_t)ev[r] < (uint32_t)a.E)
                 atomicAdd(&hist[ev[r]], 1);
             else
-                raise_error(a.err, MOE_DEV_BAD_INDEX);
+                bad = true;
         }
     }
     __syncthreads();
     block_offsets(hist, off, a.E, 0);
+    if constexpr (kDeferWrites)
+        stream_order_begin();
+    if (bad)
+        raise_error(a.err, MOE_DEV_BAD_INDEX);
     for (int32_t e = threadIdx.x; e < a.E; e += nt) {
         a.expert_count[e] = hist[e];
         a.expert_offset[e] = off[e];
@@ -255,7 +262,7 @@ struct DirectShared {
 
 // A token CTA of the direct-rank dispatch, from the expert ids on; with
 // kRowLoaded the row is already in d (else it is loaded after the ids go out).
-template <int kChunks, bool kFp8, int kK, bool kRowLoaded, bool kIdsShared>
+template <int kChunks, bool kFp8, int kK, bool kRowLoaded, bool kIdsShared, bool kDeferWrites = false>
 __device__ __forceinline__ void direct_token_cta(const FusedArgs &a, const int32_t *ids, int32_t t,
                                                  LaneData<kFusedLaneCols> (&d)[kChunks],
                                                  LaneCodes<kFusedLaneCols> (&q)[kFp8 ? kChunks : 1],
@@ -341,6 +348,7 @@ __device__ __forceinline__ void direct_token_cta(const FusedArgs &a, const int32
     __syncthreads();
 
     // 4. This token's slots: warp j adds the per-warp counts of entry j.
+    //    (With kDeferWrites they are written in 5b.)
     for (int j = warp; j < a.k; j += nwarps) {
         const uint32_t v = (int)lane < nwarps ? sh.part[lane][j] : 0u;
         const uint32_t tot = __reduce_add_sync(kFullMask, v);
@@ -350,12 +358,16 @@ __device__ __forceinline__ void direct_token_cta(const FusedArgs &a, const int32
                 const int64_t row = (int64_t)(tot & 0xffffu) + (tot >> 16);
                 if (row < a.rows_cap) {
                     s = (int32_t)row;
-                    a.recv_src[row] = (int32_t)(mine + j);
-                } else {
+                    if constexpr (!kDeferWrites)
+                        a.recv_src[row] = (int32_t)(mine + j);
+                } else if constexpr (!kDeferWrites) {
                     raise_error(a.err, MOE_DEV_CAPACITY);
+                } else {
+                    s = -2; // over capacity: flagged in 5b
                 }
             }
-            a.slot[mine + j] = s;
+            if constexpr (!kDeferWrites)
+                a.slot[mine + j] = s;
             sh.slot[j] = s;
         }
     }
@@ -370,6 +382,24 @@ __device__ __forceinline__ void direct_token_cta(const FusedArgs &a, const int32
         }
     }
     __syncthreads();
+
+    // 5b. With kDeferWrites: wait for the previous kernel, then write the slots.
+    if constexpr (kDeferWrites) {
+        stream_order_begin();
+        if ((int)threadIdx.x < a.k) {
+            const int j = threadIdx.x;
+            int32_t s = sh.slot[j];
+            if (s == -2) {
+                raise_error(a.err, MOE_DEV_CAPACITY);
+                s = -1;
+                sh.slot[j] = -1;
+            } else if (s >= 0) {
+                a.recv_src[s] = (int32_t)(mine + j);
+            }
+            a.slot[mine + j] = s;
+        }
+        __syncthreads();
+    }
 
     // 6. Payload to the k slots.
 #pragma unroll
@@ -398,6 +428,27 @@ __global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct(FusedArgs
     LaneData<kFusedLaneCols> d[kChunks];
     LaneCodes<kFusedLaneCols> q[kFp8 ? kChunks : 1];
     direct_token_cta<kChunks, kFp8, kK, false, false>(a, a.topk_idx, t, d, q, false, sh);
+}
+
+// dispatch_direct when the caller states (MOE_INPUTS_READY) that x and the
+// routing were complete before the previous kernel in the stream began: all
+// the reading and computing (ids, row, codes, counts, slots, the histogram and
+// scan) happens before waiting for that kernel, so it overlaps that kernel's
+// tail, and only the writes follow the wait (the previous kernel may still be
+// reading the buffers this one writes).
+template <int kChunks, bool kFp8, int kK>
+__global__ void __launch_bounds__(kFusedMaxThreads, 1) dispatch_direct_ready(FusedArgs a)
+{
+    extern __shared__ int32_t sm[];
+    __shared__ DirectShared<kK> sh;
+    const int32_t t = blockIdx.x;
+    if (t == a.T) {
+        direct_meta_cta<false, true>(a, a.topk_idx, sm);
+        return;
+    }
+    LaneData<kFusedLaneCols> d[kChunks];
+    LaneCodes<kFusedLaneCols> q[kFp8 ? kChunks : 1];
+    direct_token_cta<kChunks, kFp8, kK, false, false, true>(a, a.topk_idx, t, d, q, false, sh);
 }
 
 // ---- after the router (decode) ----------------------------------------------------

@@ -162,7 +162,7 @@ int check_config(const moe_config *c)
         return MOE_ERR_INVALID_ARG;
     if (c->H <= 0 || c->k <= 0 || c->E <= 0 || c->R <= 0 || c->E % c->R != 0)
         return MOE_ERR_INVALID_ARG;
-    if ((c->flags & ~(MOE_FP8 | MOE_PAD128)) != 0)
+    if ((c->flags & ~(MOE_FP8 | MOE_PAD128 | MOE_INPUTS_READY)) != 0)
         return MOE_ERR_INVALID_ARG;
     if (c->H % 8 != 0 || c->E > MOE_MAX_EXPERTS || c->k > MOE_MAX_TOPK)
         return MOE_ERR_UNSUPPORTED;
@@ -255,12 +255,28 @@ int cached_per_sm(const void *fn, int block, size_t smem)
 // 1024 threads are resident in one wave.
 // after_router: the previous kernel in the stream is the router of the same
 // moe_route_dispatch call, so the direct-rank kernel may load x before waiting.
-cudaError_t launch_small(bool fp8, int per, int32_t T, cudaStream_t s, const FusedArgs &f, bool after_router)
+// inputs_ready: the caller's MOE_INPUTS_READY (x and the routing were complete
+// before the previous kernel began), so it may read everything before waiting.
+cudaError_t launch_small(bool fp8, int per, int32_t T, cudaStream_t s, const FusedArgs &f, bool after_router,
+                         bool inputs_ready)
 {
     const bool pad = f.pad128 != 0;
     const unsigned grid = pad ? (unsigned)T : (unsigned)T + 1;
     const int32_t chunks = (f.H + chunk_cols<kFusedLaneCols>() - 1) / chunk_cols<kFusedLaneCols>();
     const unsigned block = (unsigned)((chunks + per - 1) / per * kWarp);
+    if (inputs_ready && !pad) {
+        const int i = per == 1 ? 0 : (per == 2 ? 1 : 2);
+        static const SmallKernel t[2][2][3] = {
+            {{dispatch_direct_ready<1, false, 8>, dispatch_direct_ready<2, false, 8>,
+              dispatch_direct_ready<4, false, 8>},
+             {dispatch_direct_ready<1, false, kFusedMaxK>, dispatch_direct_ready<2, false, kFusedMaxK>,
+              dispatch_direct_ready<4, false, kFusedMaxK>}},
+            {{dispatch_direct_ready<1, true, 8>, dispatch_direct_ready<2, true, 8>,
+              dispatch_direct_ready<4, true, 8>},
+             {dispatch_direct_ready<1, true, kFusedMaxK>, dispatch_direct_ready<2, true, kFusedMaxK>,
+              dispatch_direct_ready<4, true, kFusedMaxK>}}};
+        return launch(t[fp8][f.k > 8][i], grid, block, fused_smem(f.E), s, f);
+    }
     if (after_router && !pad && f.k <= 8) {
         const int i = per == 1 ? 0 : (per == 2 ? 1 : 2);
         static const SmallKernel t[2][3] = {
@@ -655,7 +671,8 @@ int run_dispatch(const moe_config *cfg, int32_t T, const void *x, const int32_t 
         f.recv_src = out->recv_src;
         f.slot = slot;
         f.err = dev_err;
-        const cudaError_t e = launch_small(fp8, per, T, s, f, after_router);
+        const cudaError_t e = launch_small(fp8, per, T, s, f, after_router,
+                                           !after_router && (cfg->flags & MOE_INPUTS_READY));
         if ((st = launched(e)) != MOE_OK)
             return st;
     } else if (use_multi(cfg, T)) {

@@ -58,6 +58,12 @@ extern "C" {
 /* moe_config.flags */
 #define MOE_FP8 1    /* payload as e4m3 codes plus one fp32 scale per 128 columns */
 #define MOE_PAD128 2 /* every expert segment padded to a multiple of 128 rows      */
+/* The caller states that x, topk_idx and topk_w were complete before the
+ * previous kernel in the stream began (that kernel does not write them): the
+ * dispatch may read and compute before waiting for it, and only its writes
+ * wait.  moe_dispatch uses it at decode sizes; other calls ignore it, and
+ * moe_route_dispatch ignores it (its ids come from its own router). */
+#define MOE_INPUTS_READY 4
 
 /* Host status codes. */
 #define MOE_OK 0

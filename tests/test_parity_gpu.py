@@ -26,10 +26,10 @@ if torch.cuda.is_available():
     import combine_route_meta_b200 as moe
 
 
-def run_gpu(x, idx, w, *, E, R, fp8, pad128=False, rows_cap=None):
+def run_gpu(x, idx, w, *, E, R, fp8, pad128=False, rows_cap=None, inputs_ready=False):
     T, H = x.shape
     k = idx.shape[1]
-    cfg = moe.make_config(H, k, E, R, fp8, pad128)
+    cfg = moe.make_config(H, k, E, R, fp8, pad128, inputs_ready)
     buf = moe.Buffers(cfg, T, "cuda", rows_cap)
     buf.recv_x.view(torch.uint8).fill_(POISON)
     if buf.recv_scale is not None:
@@ -84,9 +84,10 @@ def assert_combine_close(y_bits, ref):
     assert bad.size == 0, f"{len(bad)} elements out of tolerance, first {bad[:3]}, max err {err.max()}"
 
 
-def check_problem(x, idx, w, *, E, R, fp8, pad128=False, rows_cap=None, expect_bits=0,
+def check_problem(x, idx, w, *, E, R, fp8, pad128=False, rows_cap=None, expect_bits=0, inputs_ready=False,
                   expert_out=None):
-    buf, bits, _ = run_gpu(x, idx, w, E=E, R=R, fp8=fp8, pad128=pad128, rows_cap=rows_cap)
+    buf, bits, _ = run_gpu(x, idx, w, E=E, R=R, fp8=fp8, pad128=pad128, rows_cap=rows_cap,
+                           inputs_ready=inputs_ready)
     o = oracle.dispatch(x, idx, E=E, R=R, fp8=fp8, pad128=pad128, rows_cap=buf.rows_cap,
                         recv_fill=POISON)
     assert bits == o["err"] == expect_bits
@@ -540,3 +541,22 @@ def test_layout_then_payload_equals_the_oracle(T, H, E, R, k, fp8, pad128):
     assert moe.check() == 0
     o = oracle.dispatch(x, idx, E=E, R=R, fp8=fp8, pad128=pad128, rows_cap=buf.rows_cap, recv_fill=POISON)
     assert_dispatch_equal(dispatch_host(buf), o)
+
+
+@pytest.mark.parametrize("T,H,E,R,k,fp8,distinct,bad,cap", [
+    (128, 7168, 256, 8, 8, True, True, False, None),     # DeepSeek-V3-shaped decode
+    (128, 7168, 384, 16, 8, True, True, False, None),    # Kimi-K2-shaped decode
+    (64, 4096, 128, 8, 12, True, False, False, None),    # 16 own ids, duplicates
+    (100, 2048, 64, 4, 8, False, True, False, None),     # bf16 rows
+    (40, 1024, 32, 4, 4, True, True, True, None),        # bad ids: flagged after the wait
+    (50, 1024, 16, 4, 4, False, True, False, 120),       # capacity short of T*k
+])
+def test_inputs_ready_dispatch(T, H, E, R, k, fp8, distinct, bad, cap):
+    # MOE_INPUTS_READY: the decode kernel reads and computes before waiting for
+    # the previous kernel and writes after; the results are those of moe_dispatch
+    x, idx, w = random_problem(T + k, T, H, E, k, distinct=distinct)
+    if bad:
+        idx[3, 1] = E + 2
+        idx[T - 1, 0] = -1
+    bits = (moe.DEV_BAD_INDEX if bad else 0) | (moe.DEV_CAPACITY if cap is not None else 0)
+    check_problem(x, idx, w, E=E, R=R, fp8=fp8, rows_cap=cap, expect_bits=bits, inputs_ready=True)
