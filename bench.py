@@ -304,7 +304,7 @@ def rotating_sets(set_bytes, l2_bytes):
     return 1 if set_bytes >= 2 * l2_bytes else min(64, math.ceil(2 * l2_bytes / set_bytes) + 1)
 
 
-def config_for(w, world, rows_cap):
+def config_for(w, world, rows_cap, parallelism="replicas"):
     """The `config` object of a JSON line; both arms print the same one."""
     one_set = rotating_sets(step_set_bytes(w, rows_cap), B200_L2_BYTES) == 1
     return {"workload": w.name, "T": w.T, "H": w.H, "E": w.E, "R": w.R, "k": w.k,
@@ -314,7 +314,7 @@ def config_for(w, world, rows_cap):
                    "rotating input sets: over 2x L2 of other sets touched between uses of a set"),
             "graphs": "CUDA graphs of 8+ steps over the rotating sets, replayed back to back",
             "inputs": "written before the step; the dispatch is told so (MOE_INPUTS_READY)",
-            "parallelism": f"replicas x{world}"}
+            "parallelism": f"{parallelism} x{world}"}
 
 
 def run_gpu(args, name, rank, world, with_e2e):
@@ -538,6 +538,93 @@ def run_gpu(args, name, rank, world, with_e2e):
                 comb_ms=comb_ms, pay_ms=pay_ms, clocks=clocks, launches_per_step=launches_per_step,
                 step_kernels=step_kernels, disp_kernels=disp_kernels, e2e=e2e, nsets=nsets,
                 set_bytes=set_bytes, l2=l2, per_graph=per_graph)
+
+
+def ep_ranks_check(E, world):
+    """Expert parallelism puts E/world experts on each rank: world must divide E
+    and stay within the library's rank limit."""
+    if world < 1 or E % world != 0 or world > 64:
+        raise SystemExit(f"--parallelism ep: {world} ranks cannot share {E} experts evenly (at most 64)")
+
+
+def ep_step_bytes(w):
+    """Algorithmic bytes of one rank's expert-parallel step: its dispatch and
+    combine, as on one GPU (x read once, k rows written, k rows read back, y
+    written, and the metadata); the rows cross NVLink or stay local depending
+    on which rank hosts the expert."""
+    d, c = algorithmic_bytes(w.T, w.H, w.E, 1, w.k, w.fp8)
+    return d + c
+
+
+def run_ep(args, name, rank, world):
+    """Expert parallelism over `world` GPUs, one rank each: every rank
+    dispatches its own batch to the ranks hosting its experts and combines their
+    outputs (ExpertParallel: NCCL count exchange, peer stores, device-side
+    completion flags).  Returns the max-over-ranks device milliseconds of K steps."""
+    import dataclasses
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    import combine_route_meta_b200 as moe
+    from combine_route_meta_b200.ep import ExpertParallel
+    from workloads import WORKLOADS, make_expert_out, make_inputs
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    if not dist.is_initialized():   # one rank without torchrun
+        import socket
+        with socket.socket() as so:
+            so.bind(("127.0.0.1", 0))
+            port = so.getsockname()[1]
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                                timeout=datetime.timedelta(seconds=120))
+    w = dataclasses.replace(WORKLOADS[name], seed=WORKLOADS[name].seed + rank)
+    ep_ranks_check(w.E, world)
+    _, x, idx, wts = make_inputs(w)
+    ep = ExpertParallel(w.H, w.k, w.E, w.fp8, w.pad128, T_max=w.T, device=dev)
+    ep.expert_out.copy_(torch.from_numpy(np.ascontiguousarray(make_expert_out(w, ep.rows_cap)).view(np.int16))
+                        .to(dev).view(torch.bfloat16))
+    xd = torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).to(dev).view(torch.bfloat16)
+    idd, wd = torch.from_numpy(idx).to(dev), torch.from_numpy(wts).to(dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step():
+        dst = ep.dispatch(xd, idd, stream)
+        ep.experts_done(stream)     # the experts' kernels would run here
+        return ep.combine(idd, dst, wd, stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    ep.check(stream)
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    t_warm = time.monotonic()
+    while sampler.count() < 3 and time.monotonic() - t_warm < 5.0:
+        with torch.cuda.stream(stream):
+            for _ in range(20):
+                step()
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    sampler.mark_start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    sampler.mark_end()
+    clocks = sampler.stop()
+    ep.check(stream)
+    ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    kernels_per_step = 9   # layout, count all-gather, rows, payload, wait, signal, wait, combine (+ NCCL)
+    del ep
+    return dict(w=w, total_ms=ms, clocks=clocks, kernels_per_step=kernels_per_step)
 
 
 def summarize(r, steps, world, peak, peak_kind):
@@ -821,6 +908,9 @@ def main():
                          "under per_config (default: the other T >= 4096 configs and the decode "
                          "config when the headline is the default; 'none' for none)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--parallelism", default="replicas", choices=["replicas", "ep"],
+                    help="replicas: every rank runs its own single-GPU step; ep: the ranks form one "
+                         "expert-parallel group (rank d hosts experts [d E/N, (d+1) E/N))")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op", default=None, choices=["rank_partial", "silu_quant", "router", "route_dispatch",
                                                    "ep"],
@@ -867,7 +957,8 @@ def main():
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_for(w0, max(world, args.gpus), cap),
+            "config": config_for(w0, max(world, args.gpus), cap if args.parallelism == "replicas" else w0.T * w0.k,
+                                 args.parallelism),
             "cpu_baseline": {"value": round(g, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": round(g, 3), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -880,6 +971,28 @@ def main():
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if args.parallelism == "ep":
+        r = run_ep(args, args.workload, rank, world)
+        w = r["w"]
+        ms = r["total_ms"] / args.steps
+        step_bytes = ep_step_bytes(w)
+        line = {
+            "metric": METRIC, "value": round(job_throughput(step_bytes, world, ms), 1), "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": config_for(w, world, w.T * w.k, "ep"),
+            "total_us": round(ms * 1e3, 2), "bytes_per_step_per_rank": step_bytes,
+            "gpu_launches": r["kernels_per_step"] * args.steps * world,
+            "clocks": r["clocks"],
+            "note": "expert parallelism: rank d hosts experts [d E/N, (d+1) E/N); rows cross NVLink "
+                    "to the hosting rank; eager launches (no graph)",
+        }
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+        return
     r = run_gpu(args, args.workload, rank, world, with_e2e=True)
     head = summarize(r, args.steps, world, peak, peak_kind)
     w = r["w"]

@@ -10,6 +10,7 @@ import socket
 import subprocess
 import sys
 
+import pytest
 import torch.multiprocessing as mp
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -106,3 +107,31 @@ def test_expert_parallel_count_exchange_two_gloo_ranks():
         assert p.exitcode == 0
     want = [[i * (r + 1) for i in range(8)] for r in range(2)]
     assert out[0] == want and out[1] == want
+
+
+def test_expert_parallel_bench_plumbing():
+    # the host-side parts of `bench.py --parallelism ep`: which rank counts can
+    # share the experts, the per-rank byte model, and the config both arms print
+    sys.path.insert(0, ROOT)
+    import bench
+    from workloads import WORKLOADS
+    for n in (1, 2, 4, 8):
+        bench.ep_ranks_check(256, n)
+    for bad in (3, 0, 128):
+        with pytest.raises(SystemExit):
+            bench.ep_ranks_check(256, bad)
+    w = WORKLOADS["dsv3_decode"]
+    d, c = bench.algorithmic_bytes(w.T, w.H, w.E, 1, w.k, w.fp8)
+    assert bench.ep_step_bytes(w) == d + c
+    cfg = bench.config_for(w, 8, w.T * w.k, "ep")
+    assert cfg["parallelism"] == "ep x8" and cfg["workload"] == "dsv3_decode"
+
+
+def test_reference_arm_prints_the_ep_config():
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "3",
+                        "--workload", "tiny", "--parallelism", "ep"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["config"]["parallelism"] == "ep x1"
