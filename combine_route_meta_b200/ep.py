@@ -49,6 +49,8 @@ def share_buffers(tensors, group=None):
     rank's own at its index), the others opened through CUDA IPC."""
     from torch.multiprocessing.reductions import reduce_tensor
     rank, W = dist.get_rank(group), dist.get_world_size(group)
+    if W == 1:
+        return [[t] for t in tensors]
     handles = [None] * W
     dist.all_gather_object(handles, [reduce_tensor(t) for t in tensors], group=group)
     out = []
