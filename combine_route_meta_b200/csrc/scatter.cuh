@@ -18,7 +18,7 @@
 //  - fp8: lane l owns L consecutive columns, 128/L lanes make one 128-column
 //    block; the block's |x| maximum is reduced with butterfly shuffles inside
 //    those lanes, the scale is amax/448 and each code is e4m3(x/scale) with
-//    the binary32 quotient correctly rounded (see product_decides_code) and a
+//    the binary32 quotient correctly rounded (see quantise_floats) and a
 //    saturating round-to-nearest-even conversion.  A lane stores its L codes
 //    with one L-byte store, and lane 0 stores the warp's L/4 block scales with
 //    one store when the scale row allows it.
@@ -64,29 +64,20 @@ struct LaneData {
     uint4 v[kLaneCols / 8];
 };
 
-// x / scale as the e4m3 conversion needs it.  The codes must equal those of the
-// correctly rounded binary32 quotient.  With recip = RN(1/scale), the product
-// q = RN(x * recip) lies within 2.5 units in the last place of RN(x / scale)
-// (two relative roundings of 2^-24 each, plus the half unit of RN itself).
-// e4m3 rounding is monotone and its rounding boundaries in the normal range
-// are the values whose 20 low mantissa bits are exactly 0x80000 (halfway
-// between two 3-bit mantissas).  So when q is in the e4m3 normal range
-// (>= 2^-6) and more than 3 units from such a boundary, both quotients give
-// the same code and q is used; otherwise (near a boundary, in the e4m3
-// subnormal range, a zero, or a block whose scale is below FLT_MIN) the exact
-// division is taken.  On N(0,1) data the exact branch is rare (~1e-4 of the
-// values), so it is taken once per warp when any lane needs it.
-__device__ __forceinline__ bool product_decides_code(float q)
-{
-    const uint32_t b = __float_as_uint(q) & 0x7fffffffu;
-    const uint32_t off_mid = ((b & 0xfffffu) - 0x7fffdu) & 0xfffffu; // <= 6: within 3 units of 0x80000
-    return b >= 0x3c800000u && off_mid > 6u;
-}
-
 // e4m3 codes (element 0 in the lowest byte) and the block scale of kLaneCols
 // binary32 values per lane; the 128/kLaneCols lanes of a 128-column block
 // reduce the maximum together.  All lanes of the warp call this (inactive lanes
 // hold zeros).  An all-zero block gets scale 0 and +0 codes.
+//
+// The codes must equal those of the correctly rounded quotient Q = RN(x/scale).
+// With r = RN(1/scale), the real product P = x r is within a relative 2^-24 of
+// x/scale, so Q lies within P(1 +- 2^-23).  The codes of RN(x RN(r(1 - 2^-20)))
+// and RN(x RN(r(1 + 2^-20))) bracket it: those two products lie within a
+// relative 2^-23 of P(1 -+ 2^-20), outside P(1 +- 2^-23) on either side, and
+// e4m3 rounding (nearest, ties to even, saturating) never decreases.  Where the
+// two codes agree they are Q's code.  Four codes are compared at once; the rare
+// group where they differ (a quotient near an e4m3 rounding boundary), and a
+// block whose scale is below FLT_MIN (r not finite), takes the exact division.
 template <int kLaneCols>
 __device__ __forceinline__ void quantise_floats(const float (&f)[kLaneCols],
                                                 uint32_t (&codes)[kLaneCols / 4], float &scale_out)
@@ -101,25 +92,33 @@ __device__ __forceinline__ void quantise_floats(const float (&f)[kLaneCols],
     const bool nonzero = amax > 0.0f;
     const float scale = __fdiv_rn(nonzero ? amax : 448.0f, 448.0f);
     const float recip = __frcp_rn(scale);
+    const float r_lo = recip * (1.0f - 0x1p-20f), r_hi = recip * (1.0f + 0x1p-20f);
     const bool fast = scale >= 0x1p-126f; // recip finite, products in range
-    float q[kLaneCols];
-    bool exact = !fast;
+    uint32_t undecided = fast ? 0u : 0xffffffffu; // bit i: group of 4 values i
 #pragma unroll
-    for (int i = 0; i < kLaneCols; ++i) {
-        q[i] = f[i] * recip;
-        exact |= !product_decides_code(q[i]);
+    for (int i = 0; i < kLaneCols / 4; ++i) {
+        const float *g = f + 4 * i;
+        const uint32_t lo = pack_e4m3x2(g[0] * r_lo, g[1] * r_lo) | (pack_e4m3x2(g[2] * r_lo, g[3] * r_lo) << 16);
+        const uint32_t hi = pack_e4m3x2(g[0] * r_hi, g[1] * r_hi) | (pack_e4m3x2(g[2] * r_hi, g[3] * r_hi) << 16);
+        codes[i] = lo;
+        undecided |= lo != hi ? 1u << i : 0u;
     }
-    if (__any_sync(kFullMask, nonzero && exact)) {
+    if (!nonzero)
+        undecided = 0;
+    if (__any_sync(kFullMask, undecided != 0)) {
 #pragma unroll
-        for (int i = 0; i < kLaneCols; ++i)
-            if (!fast || !product_decides_code(q[i]))
-                q[i] = __fdiv_rn(f[i], scale);
+        for (int i = 0; i < kLaneCols / 4; ++i)
+            if ((undecided >> i) & 1u) {
+                const float *g = f + 4 * i;
+                codes[i] = pack_e4m3x2(__fdiv_rn(g[0], scale), __fdiv_rn(g[1], scale)) |
+                           (pack_e4m3x2(__fdiv_rn(g[2], scale), __fdiv_rn(g[3], scale)) << 16);
+            }
     }
+    if (!nonzero) {
 #pragma unroll
-    for (int i = 0; i < kLaneCols / 4; ++i)
-        codes[i] = nonzero ? pack_e4m3x2(q[4 * i + 0], q[4 * i + 1]) |
-                                 (pack_e4m3x2(q[4 * i + 2], q[4 * i + 3]) << 16)
-                           : 0u;
+        for (int i = 0; i < kLaneCols / 4; ++i)
+            codes[i] = 0u;
+    }
     scale_out = nonzero ? scale : 0.0f;
 }
 
