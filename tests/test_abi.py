@@ -64,8 +64,11 @@ def test_config_validation_statuses():
         sizes = moe.moe_dispatch_sizes()
         assert moe.moe_dispatch_sizes_for(ctypes.byref(cfg), 4, 32, ctypes.byref(sizes)) == want
         assert moe.moe_rows_capacity(ctypes.byref(cfg), 4) == -1
-    cfg = moe.moe_config(128, 2, 8, 2, 4)  # unknown flag bit
-    assert moe.moe_rows_capacity(ctypes.byref(cfg), 4) == -1
+    for bit in (8, 1 << 30):  # flag bits the header does not define
+        cfg = moe.moe_config(128, 2, 8, 2, bit)
+        assert moe.moe_rows_capacity(ctypes.byref(cfg), 4) == -1
+    cfg = moe.moe_config(128, 2, 8, 2, moe.INPUTS_READY)
+    assert moe.moe_rows_capacity(ctypes.byref(cfg), 4) > 0
 
 
 def test_dispatch_rejects_bad_arguments_before_touching_the_gpu():

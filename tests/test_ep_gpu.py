@@ -300,3 +300,15 @@ def test_expert_parallel_host_flow_on_a_one_rank_group():
     r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True,
                        timeout=300)
     assert "ONE RANK OK" in r.stdout, r.stdout[-2000:] + r.stderr[-4000:]
+
+
+def test_bench_expert_parallel_mode_on_one_rank():
+    # `bench.py --parallelism ep` as a one-rank group: the graph-replayed EP step
+    # runs, checks the device error word and prints its JSON line
+    import json
+    r = subprocess.run([sys.executable, "bench.py", "--parallelism", "ep", "--workload", "dsv3_decode",
+                        "--steps", "5", "--warmup", "3"], cwd=ROOT, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["config"]["parallelism"] == "ep x1" and line["value"] > 0 and line["steps"] == 5
