@@ -260,6 +260,27 @@ struct DirectShared {
     int32_t own[kK];
 };
 
+// fp8 rows of the direct-rank dispatch leave as whole-row bulk stores (one per
+// slot for the codes, one for the scales) from a shared-memory copy of the row,
+// when the row fits it and both stores are whole 16-byte units (H % 512 == 0
+// makes the H/32 scale bytes one).  One contiguous multi-kilobyte write per
+// receive row is what the HBM write stream favours; the register path writes
+// every slot's row in 256-byte pieces from all warps.
+constexpr int32_t kDirectBulkMaxH = 8192;
+
+__host__ __device__ inline bool direct_bulk_rows(int32_t H) { return H % 512 == 0 && H <= kDirectBulkMaxH; }
+
+struct __align__(128) DirectRow {
+    uint8_t b[kDirectBulkMaxH + kDirectBulkMaxH / 32]; // codes, then the H/128 fp32 scales
+};
+
+// The CTA's shared-memory row (allocated only in kernels that use it).
+__device__ __forceinline__ DirectRow &sh_row()
+{
+    __shared__ DirectRow row;
+    return row;
+}
+
 // A token CTA of the direct-rank dispatch, from the expert ids on; with
 // kRowLoaded the row is already in d (else it is loaded after the ids go out).
 template <int kChunks, bool kFp8, int kK, bool kRowLoaded, bool kIdsShared, bool kDeferWrites = false>
@@ -372,13 +393,30 @@ __device__ __forceinline__ void direct_token_cta(const FusedArgs &a, const int32
         }
     }
 
-    // 5. The row's codes (unless already made), while the slot sums above complete.
+    // 5. The row's codes (unless already made), while the slot sums above
+    //    complete; for the bulk stores they go to the shared-memory row.
+    const bool bulk_rows = kFp8 && direct_bulk_rows(a.H);
     if constexpr (kFp8) {
         if (!quantised) {
 #pragma unroll
             for (int i = 0; i < kChunks; ++i)
                 if (warp + i * nwarps < chunks)
                     quantise_lane<L>(d[i], q[i].codes, q[i].scale);
+        }
+        if (bulk_rows) {
+            static_assert(L == 8, "two code words per lane");
+            uint8_t *row = sh_row().b;
+#pragma unroll
+            for (int i = 0; i < kChunks; ++i) {
+                const int32_t c = warp + i * nwarps;
+                const int32_t col = c * chunk_cols<L>() + (int32_t)lane * L;
+                if (c < chunks) { // H % 512 == 0: every column of the chunk is in the row
+                    *reinterpret_cast<uint2 *>(row + col) = make_uint2(q[i].codes[0], q[i].codes[1]);
+                    if ((lane & 15) == 0) // the first lane of each 128-column block
+                        reinterpret_cast<float *>(row + a.H)[col / 128] = q[i].scale;
+                }
+            }
+            fence_async_shared(); // the bulk stores read what the generic proxy wrote
         }
     }
     __syncthreads();
@@ -401,7 +439,26 @@ __device__ __forceinline__ void direct_token_cta(const FusedArgs &a, const int32
         __syncthreads();
     }
 
-    // 6. Payload to the k slots.
+    // 6. Payload to the k slots: thread j issues slot j's two bulk stores and
+    //    waits until they have read the row (the writes complete with the grid),
+    //    or every warp stores its chunks from registers.
+    if constexpr (kFp8) {
+        if (bulk_rows) {
+            if ((int)threadIdx.x < a.k) {
+                const int32_t s = sh.slot[threadIdx.x]; // -1 or a row below rows_cap
+                const uint8_t *row = sh_row().b;
+                if (s >= 0) {
+                    bulk_store(static_cast<uint8_t *>(a.recv_x) + (int64_t)s * a.H, smem_addr(row),
+                               (uint32_t)a.H);
+                    bulk_store(a.recv_scale + (int64_t)s * (a.H / 128), smem_addr(row + a.H),
+                               (uint32_t)(a.H / 32));
+                }
+                bulk_commit();
+                bulk_wait_read<0>();
+            }
+            return;
+        }
+    }
 #pragma unroll
     for (int i = 0; i < kChunks; ++i) {
         const int32_t c = warp + i * nwarps;
