@@ -75,7 +75,10 @@ def source_digest():
     d = hashlib.sha256()
     src = os.path.join(HERE, "combine_route_meta_b200", "csrc")
     for name in sorted(os.listdir(src)):
-        with open(os.path.join(src, name), "rb") as f:
+        path = os.path.join(src, name)
+        if not os.path.isfile(path):
+            continue
+        with open(path, "rb") as f:
             d.update(name.encode() + b"\0" + f.read())
     return d.hexdigest()[:16]
 

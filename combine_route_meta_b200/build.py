@@ -33,7 +33,7 @@ NVCC_FLAGS = [
 def _inputs():
     files = list(SOURCES)
     for d in (CSRC, INCLUDE):
-        files += [os.path.join(d, f) for f in os.listdir(d) if f.endswith((".cuh", ".h"))]
+        files += [os.path.join(d, f) for f in os.listdir(d) if f.endswith((".cuh", ".h", ".inc"))]
     return files
 
 

@@ -1,6 +1,7 @@
 // C ABI of the MoE dispatch / combine library: host-side validation and
 // launches.  The declarations and their contracts are in
 // include/moe_dispatch_combine.h.
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <atomic>
@@ -54,7 +55,7 @@ struct DeviceInfo {
     std::atomic<bool> ready{false};
     int sms = 0;
     // resident CTAs per SM of the kernels whose grid is one wave
-    int silu_per_sm = 1;
+    int silu_per_sm[2] = {1, 1}; // silu_quant_rows<1>, <kSiluWideCtas>
     int router_per_sm[4] = {1, 1, 1, 1}; // 4, 8, 16, 32 logits per lane
     int send_per_sm[2] = {1, 1};         // combine_partial_send<false>, <true>
     int recv_per_sm = 1;
@@ -98,7 +99,8 @@ int device_info(DeviceInfo **out)
                                  (int)kBulkMaxSmem) != cudaSuccess)
             return MOE_ERR_CUDA;
         const int rb = kRouterWarps * kWarp;
-        if (!(d.silu_per_sm = resident_per_sm(silu_quant_rows, kSiluThreads, 0)) ||
+        if (!(d.silu_per_sm[0] = resident_per_sm(silu_quant_rows<1>, kSiluThreads, 0)) ||
+            !(d.silu_per_sm[1] = resident_per_sm(silu_quant_rows<kSiluWideCtas>, kSiluThreads, 0)) ||
             !(d.router_per_sm[0] = resident_per_sm(router_topk<4>, rb, 0)) ||
             !(d.router_per_sm[1] = resident_per_sm(router_topk<8>, rb, 0)) ||
             !(d.router_per_sm[2] = resident_per_sm(router_topk<16>, rb, 0)) ||
@@ -892,9 +894,15 @@ int moe_silu_quant(int64_t rows_cap, int32_t I, const void *gate_up, const int32
     a.act = static_cast<uint8_t *>(act);
     a.scale = act_scale;
     a.col_major = scale_col_major ? 1 : 0;
-    // A fixed grid, whatever the routing: the kernel reads how many rows are in use.
-    const unsigned grid = (unsigned)(dev->sms * dev->silu_per_sm);
-    return launched(launch(silu_quant_rows, grid, kSiluThreads, 0, static_cast<cudaStream_t>(stream), a));
+    // A fixed grid, whatever the routing (the kernel reads how many rows are in
+    // use); the build and the grid follow the buffer's capacity in 512-column units.
+    const int64_t units_cap = rows_cap * ((I + 511) / 512);
+    const int64_t wide = (int64_t)dev->sms * dev->silu_per_sm[1];
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (units_cap >= wide * (kSiluThreads / kWarp) * kSiluUnitsPerWarpWide)
+        return launched(launch(silu_quant_rows<kSiluWideCtas>, (unsigned)wide, kSiluThreads, 0, s, a));
+    const unsigned grid = (unsigned)(dev->sms * std::min(dev->silu_per_sm[0], kSiluNarrowCtas));
+    return launched(launch(silu_quant_rows<1>, grid, kSiluThreads, 0, s, a));
 }
 
 int moe_silu_mul(int64_t n, const void *gate, const void *up, float *act, double *fast_value,
