@@ -89,7 +89,7 @@ def _silu_problem(rows, I, seed, pad_frac=0.2):
 
 @pytest.mark.parametrize("rows,I,in_use,col_major", [(1024, 2048, 1000, False), (1024, 2048, 1024, True),
                                                      (300, 384, 299, False), (70, 1152, 0, False),
-                                                     (4096, 2048, 4000, True)])
+                                                     (4096, 2048, 4000, True), (8192, 1024, 8000, False)])
 def test_silu_quant_bit_exact(rows, I, in_use, col_major):
     gu, src = _silu_problem(rows, I, rows + I)
     act_ref, sc_ref = oracle.silu_quant(gu, src, in_use, col_major=col_major, fill=0xA5)
