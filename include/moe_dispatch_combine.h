@@ -299,13 +299,15 @@ MOE_API int moe_silu_quant(int64_t rows_cap, int32_t I, const void *gate_up,
  * the binary32 number nearest to g u / (1 + e^-g) for g = gate[i], u = up[i]
  * (bf16 device arrays; "Lower latency and higher throughput with multi-node
  * DeepSeek deployment", section "Quantização": SiLU of the gate times up, the
- * input of the block quantiser).  The kernel evaluates g u sigmoid(g) in fp64
- * (sigmoid from a per-CTA table for common gates) and certifies the rounding,
- * falling back to double-double arithmetic near a binary32 rounding boundary;
- * exact_only != 0 takes the double-double tier for every value.  fast_value (fp64 device, may be NULL) receives the fp64 value of the
- * first tier for each pair (meaningful for finite, nonzero, normal inputs
- * with gate >= -200), for checking its error bound.  act is fp32 device.
- * n = 0 launches nothing.  Returns a status.
+ * input of the block quantiser).  The kernel takes the same three tiers as
+ * moe_silu_quant: for common gates a binary32 product with a table of silu(g)
+ * as a pair of binary32 numbers (made at build time) and a certified rounding,
+ * else g u sigmoid(g) in fp64 with a certified rounding, and double-double
+ * arithmetic near a binary32 rounding boundary; exact_only != 0 takes the
+ * double-double tier for every value.  fast_value (fp64 device, may be NULL)
+ * receives the fp64 tier's value for each pair (meaningful for finite,
+ * nonzero, normal inputs with gate >= -200), for checking its error bound.
+ * act is fp32 device.  n = 0 launches nothing.  Returns a status.
  */
 MOE_API int moe_silu_mul(int64_t n, const void *gate, const void *up, float *act,
                          double *fast_value, int32_t exact_only, void *stream);
