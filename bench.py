@@ -496,44 +496,83 @@ def run_gpu(args, name, rank, world, with_e2e):
 
     e2e = None
     if with_e2e:
-        # End to end through the public API with host buffers: H2D of the step's
-        # inputs, dispatch, combine, D2H of y, every step.
-        st = sets[0]
+        # End to end through the public API with host buffers, every step: H2D
+        # of the step's inputs from pinned memory, dispatch, combine, D2H of y.
+        # Steady state of a stream of batches: two device sets, the uploads on
+        # one copy stream and the downloads on another, so step i's result goes
+        # down while step i+1's inputs come up (the host link is full duplex)
+        # and the kernels run between them.  Events order the reuse of a set.
         pin = dict(pin_memory=True)
         x_h = torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).pin_memory()
         idx_h = torch.from_numpy(idx).pin_memory()
         w_h = torch.from_numpy(wts).pin_memory()
         eo_h = (None if eo_host is None else
                 torch.from_numpy(np.ascontiguousarray(eo_host).view(np.int16)).view(torch.bfloat16).pin_memory())
-        y_h = torch.empty((w.T, w.H), dtype=torch.bfloat16, **pin)
+        pipe = [sets[0]]
+        if len(sets) > 1:
+            pipe.append(sets[1])
+        else:
+            st2 = Set()
+            st2.buf = moe.Buffers(cfg, w.T, dev)
+            st2.x, st2.idx, st2.w = torch.empty_like(sets[0].x), torch.empty_like(sets[0].idx), \
+                torch.empty_like(sets[0].w)
+            st2.eo = st2.buf.recv_x if eo_host is None else torch.empty_like(sets[0].eo)
+            st2.y = torch.empty_like(sets[0].y)
+            pipe.append(st2)
+        y_h = [torch.empty((w.T, w.H), dtype=torch.bfloat16, **pin) for _ in pipe]
         h2d = x_h.numel() * 2 + idx_h.numel() * 4 + w_h.numel() * 4 + (0 if eo_h is None else eo_h.numel() * 2)
-        d2h = y_h.numel() * 2
-        e2e_steps = max(3, min(args.steps, 20))
-        e2e_ms = []
-        if dist is not None:
-            dist.barrier()  # every rank's copies share the node's host links while timed
-        for i in range(args.warmup + e2e_steps):
-            with torch.cuda.stream(stream):
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
+        d2h = y_h[0].numel() * 2
+        s_up, s_down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        up_done = [torch.cuda.Event() for _ in pipe]
+        comp_done = [torch.cuda.Event() for _ in pipe]
+        down_done = [torch.cuda.Event() for _ in pipe]
+        for b in range(len(pipe)):  # every event recorded once before its first wait
+            for ev in (up_done[b], comp_done[b], down_done[b]):
+                ev.record(stream)
+
+        def e2e_step(i):
+            b = i % len(pipe)
+            st = pipe[b]
+            with torch.cuda.stream(s_up):
+                s_up.wait_event(comp_done[b])     # the set's previous step has read its inputs
                 st.x.copy_(x_h, non_blocking=True)
                 st.idx.copy_(idx_h, non_blocking=True)
                 st.w.copy_(w_h, non_blocking=True)
                 if eo_h is not None:
                     st.eo.copy_(eo_h, non_blocking=True)
-                do_dispatch(st)
-                do_combine(st)
-                y_h.copy_(st.y, non_blocking=True)
-                e1.record(stream)
-            e1.synchronize()
-            if i >= args.warmup:
-                e2e_ms.append(e0.elapsed_time(e1))
-        e2e_med_ms = statistics.median(e2e_ms)
+                up_done[b].record(s_up)
+            stream.wait_event(up_done[b])
+            stream.wait_event(down_done[b])       # the set's previous y has gone down
+            do_dispatch(st)
+            do_combine(st)
+            comp_done[b].record(stream)
+            with torch.cuda.stream(s_down):
+                s_down.wait_event(comp_done[b])
+                y_h[b].copy_(st.y, non_blocking=True)
+                down_done[b].record(s_down)
+
+        e2e_steps = max(3, min(args.steps, 20))
+        for i in range(args.warmup):
+            e2e_step(i)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()  # every rank's copies share the node's host links while timed
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s_up)
+        for i in range(e2e_steps):
+            e2e_step(args.warmup + i)
+        s_down.wait_stream(s_up)
+        s_down.wait_stream(stream)
+        e1.record(s_down)
+        e1.synchronize()
+        e2e_med_ms = e0.elapsed_time(e1) / e2e_steps
         if dist is not None:
             e2e_med_ms = max_over_ranks(e2e_med_ms, dist, dev)
+        torch.cuda.synchronize()
         if moe.check(stream) != 0:
             raise RuntimeError("device error during the end-to-end steps")
         e2e = dict(ms=e2e_med_ms, h2d=h2d, d2h=d2h)
+        del pipe
 
     sets.clear()
     torch.cuda.synchronize()
@@ -1019,7 +1058,9 @@ def main():
                                 "pct_of_spec_peak", "bytes_per_step", "step_us_spread", "roofline")},
         "e2e": {"value": round(job_throughput(step_bytes, world, e2e["ms"]), 3), "unit": "GB/s",
                 "h2d_bytes_per_step": e2e["h2d"] * world, "d2h_bytes_per_step": e2e["d2h"] * world,
-                "ms_per_step": round(e2e["ms"], 4)},
+                "ms_per_step": round(e2e["ms"], 4),
+                "copies": ("pinned host buffers; inputs up on one stream, y down on another, two "
+                           "device sets, so one step's download overlaps the next step's upload")},
         "kernels_per_step": head["kernels_per_step"],
         "timing": head["timing"],
         "clocks": head["clocks"],
